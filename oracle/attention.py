@@ -1,0 +1,105 @@
+"""O1 - sink + window + own-chunk attention, written as its plain definition.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+What is computed, and where the pages fix it:
+
+* Generation is chunk-level causal autoregression: chunk c is produced from the
+  chunks before it, whose self-attention K/V sit in the KV cache
+  (LongLive explainer, dpshk.com, sec. 二; LongLive-2.0 explainer, wmrh.cn, sec. 3).
+* Keys visible to the queries of chunk c
+    - the own chunk, with full attention inside it; nothing from a later chunk
+      (LongLive-2.0 explainer, sec. 6: a noisy chunk sees the clean earlier
+      chunks and itself, never the future);
+    - the frame sink: the first S latent frames, kept for the whole rollout
+      (dpshk.com sec. 六; techwalker.com LONGLIVE article, sec. 四 and 六);
+    - the short window: the most recent W latent frames before the chunk, older
+      ones evicted (dpshk.com sec. 五; techwalker.com sec. 四 and 六: chunk 3,
+      window 9, sink = first 3 latent frames).
+  A frame below S is a sink frame only; the window is the last W frames that
+  precede the chunk and are not sink frames.
+* Attention itself: o_i = sum_j softmax_j(q_i . k_j / sqrt(D)) v_j over the
+  visible keys j, per head. The 1/sqrt(D) scale is the standard scaled
+  dot-product scale; the pages print no other.
+
+The mask is built over the full token history (frame f_j = j // T of every key
+token j), not over cache slots: the oracle knows nothing about the ring buffer.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def frame_visible(query_frame: int, key_frame: int, S: int, W: int, F: int) -> bool:
+    """Is key frame `key_frame` visible to a query in frame `query_frame`?"""
+    cq = query_frame // F
+    ck = key_frame // F
+    if ck == cq:
+        return True            # own chunk: full attention inside the chunk
+    if ck > cq:
+        return False           # a later chunk: never visible
+    if key_frame < S:
+        return True            # frame sink
+    return key_frame >= cq * F - W   # one of the last W frames before the chunk
+
+
+def visible_key_frames(chunk: int, S: int, W: int, F: int) -> list[int]:
+    """Sorted list of the frames whose keys the queries of `chunk` see."""
+    return [f for f in range((chunk + 1) * F) if frame_visible(chunk * F, f, S, W, F)]
+
+
+def key_mask(chunk: int, query_rows: np.ndarray, n_key_tokens: int, S: int, W: int, F: int, T: int) -> np.ndarray:
+    """Explicit boolean mask [len(query_rows)][n_key_tokens].
+
+    query_rows are token indices inside the chunk (0..F*T-1); key token j belongs
+    to frame j // T of the history.
+    """
+    q_frame = chunk * F + np.asarray(query_rows) // T           # [R]
+    k_frame = np.arange(n_key_tokens) // T                        # [N]
+    cq = (q_frame // F)[:, None]
+    ck = (k_frame // F)[None, :]
+    kf = k_frame[None, :]
+    own = ck == cq
+    past = ck < cq
+    sink = kf < S
+    window = kf >= cq * F - W
+    return own | (past & (sink | window))
+
+
+def sink_window_attention(q_bits: np.ndarray, k_hist_bits: np.ndarray, v_hist_bits: np.ndarray,
+                          chunk: int, S: int, W: int, F: int, T: int,
+                          rows=None, row_block: int = 256) -> np.ndarray:
+    """Attention output of chunk `chunk` in fp64.
+
+    q_bits       [F*T][H][D] bf16 bits, the chunk's queries
+    k_hist_bits  [(chunk+1)*F*T][H][D] bf16 bits: K of every frame generated so far,
+                 in generation order, the current chunk's K last (its k_cur)
+    v_hist_bits  same for V
+    rows         optional subset of query rows (token index in the chunk)
+    returns      [len(rows)][H][D] float64
+    """
+    Tq, H, D = q_bits.shape
+    assert Tq == F * T
+    n_keys = k_hist_bits.shape[0]
+    assert n_keys == (chunk + 1) * F * T, "history must hold every frame up to the current chunk"
+    rows = np.arange(Tq) if rows is None else np.asarray(rows)
+    out = np.empty((len(rows), H, D), dtype=np.float64)
+    scale = 1.0 / np.sqrt(D)
+    for h in range(H):
+        k = _bf16_to_f64(k_hist_bits[:, h, :])                      # [N][D]
+        v = _bf16_to_f64(v_hist_bits[:, h, :])
+        for r0 in range(0, len(rows), row_block):
+            rr = rows[r0:r0 + row_block]
+            q = _bf16_to_f64(q_bits[rr, h, :])                      # [R][D]
+            mask = key_mask(chunk, rr, n_keys, S, W, F, T)          # [R][N]
+            s = (q @ k.T) * scale
+            s = np.where(mask, s, -np.inf)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p = p / p.sum(axis=1, keepdims=True)
+            out[r0:r0 + len(rr), h, :] = p @ v
+    return out
