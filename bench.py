@@ -1,0 +1,419 @@
+"""Benchmark of the sink + window chunk-attention hot path on B200.
+
+One step = one steady-state chunk-step of the 30-layer Wan-1.3B-shaped stack:
+for every layer, ll_attn_sink_window (12 heads, head_dim 128, 4680 queries over
+3 sink + 9 window cached frames + the own 3-frame chunk = 23400 keys) followed
+by ll_kv_append of the chunk. The KV-recache of all 30 layers (sink + window,
+12 frames) is timed in the same run and reported beside the step.
+
+Prints ONE JSON line (rank 0). Multi-GPU runs (torchrun) are independent
+replicas, one video stream per GPU, with no collective on the data path
+(weak scaling); only the timing uses a MAX all-reduce.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (fp64 numpy) on a bounded sample of the
+same workload on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sink+window chunk-attention TFLOP/s & % BF16 peak; ms/chunk-step (30 layers)"
+UNIT = "TFLOP/s"
+# Wan-1.3B-shaped stack
+L, H, D, T, F, S, W = 30, 12, 128, 1560, 3, 3, 9
+TQ = F * T
+NK = (S + W + F) * T                       # visible keys in steady state: 23400
+ATTN_FLOP = 4.0 * TQ * NK * D * H          # per layer: QK^T and PV over visible keys only
+APPEND_BYTES = 2 * 2 * TQ * H * D * 2      # K and V, read + write
+RECACHE_BYTES = 2 * 2 * L * (S + W) * T * H * D * 2
+ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out + cached K, V
+# ncu DRAM traffic of one attention launch at this shape and the kernel sources it
+# was taken with (profiles/attn_sink_window_wan1.3b.md); reported only while the
+# kernel is unchanged.
+ATTN_TRAFFIC = None
+ATTN_TRAFFIC_SRC_SHA = None
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["bf16_tflops"]), float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+def _kernel_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("attn_sink_window.cuh", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "kv_cache_attention_ll_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            import torch
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_oracle_sample(seconds_target: float = 12.0):
+    """Times the CPU oracle on a bounded sample of the workload: sampled query
+    rows of one steady-state layer-chunk (all 12 heads, all 23400 visible keys).
+    Returns (TFLOP/s, sample description, threads, seconds)."""
+    import numpy as np
+    import oracle
+    from seeded_inputs import chunk_qkv
+    c = 4                                    # p = 12 = S + W: the cache is full
+    hk, hv = [], []
+    for cc in range(c + 1):
+        q, k, v = chunk_qkv(1, 0, cc, TQ, H, D)
+        hk.append(k)
+        hv.append(v)
+    kh, vh = np.concatenate(hk), np.concatenate(hv)
+    rng = np.random.default_rng(5)
+    rows = np.sort(rng.choice(TQ, 16, replace=False))
+    t0 = time.perf_counter()
+    oracle.sink_window_attention(q, kh, vh, c, S, W, F, T, rows=rows)
+    dt = time.perf_counter() - t0
+    n = int(max(16, min(TQ, 16 * seconds_target / max(dt, 1e-3))))
+    rows = np.sort(rng.choice(TQ, n, replace=False))
+    t0 = time.perf_counter()
+    oracle.sink_window_attention(q, kh, vh, c, S, W, F, T, rows=rows)
+    dt = time.perf_counter() - t0
+    flop = 4.0 * n * NK * D * H
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    desc = (f"fp64 numpy oracle, {n} of {TQ} query rows x {H} heads of one steady-state layer-chunk "
+            f"({NK} visible keys), {dt:.1f} s")
+    return flop / dt / 1e12, desc, threads, dt
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    vals = []
+    desc = threads = None
+    for i in range(args.warmup + args.steps):
+        v, desc, threads, _ = cpu_oracle_sample(seconds_target=max(2.0, 60.0 / (args.warmup + args.steps)))
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.mean(vals)
+    flop_step = ATTN_FLOP * L
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": flop_step / (value * 1e12) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "wan1.3b-30layer-chunk-step (CPU oracle on sampled query rows)", "layers": L,
+                   "heads": H, "head_dim": D, "tokens_per_frame": T, "frames_per_chunk": F,
+                   "sink_frames": S, "window_frames": W, "visible_keys": NK},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+    import kv_cache_attention_ll_b200 as ll
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    peak_tf, peak_gbs, peak_kind = _peaks()
+    g = torch.Generator(device=dev)
+    g.manual_seed(20261202 + 7919 * rank)
+
+    def randn(*shape):
+        return torch.randn(*shape, device=dev, dtype=torch.float32, generator=g).to(torch.bfloat16)
+
+    # per-layer activations of one chunk (values do not affect the runtime)
+    qs = [randn(TQ, H, D) for _ in range(L)]
+    ks = [randn(TQ, H, D) for _ in range(L)]
+    vs = [randn(TQ, H, D) for _ in range(L)]
+    outs = [torch.empty(TQ, H, D, device=dev, dtype=torch.bfloat16) for _ in range(L)]
+    kn = randn(L, (S + W) * T, H, D)
+    vn = randn(L, (S + W) * T, H, D)
+    cache = ll.ll_kv_cache_create(L, H, D, T, F, S, W)
+    # fill the cache to steady state: (S + W) / F chunks of history
+    for c in range((S + W + F - 1) // F + 1):
+        for l in range(L):
+            ll.ll_kv_append(cache, l, ks[l], vs[l], stream)
+    torch.cuda.synchronize(dev)
+    assert ll.ll_kv_cache_info(cache, 0)[0] >= S + W
+
+    # one start/end event pair around every attention launch of every timed step
+    attn_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+               for _ in range(args.steps)]
+
+    def step(ev=None):
+        for l in range(L):
+            if ev is not None:
+                ev[l][0].record(stream)
+            ll.ll_attn_sink_window(qs[l], ks[l], vs[l], cache, l, outs[l], stream)
+            if ev is not None:
+                ev[l][1].record(stream)
+            ll.ll_kv_append(cache, l, ks[l], vs[l], stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    _barrier(world)
+
+    # ---- device-timed steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize(dev)
+        _barrier(world)
+        e0.record(stream)
+        for i in range(args.steps):
+            step(attn_ev[i])
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    total_ms = e0.elapsed_time(e1)
+    attn_ms = [a.elapsed_time(b) for ev in attn_ev for a, b in ev]
+    _barrier(world)
+    total_ms = _max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    value = world * ATTN_FLOP * L / (ms_step * 1e-3) / 1e12
+
+    # ---- dominant kernel: attention, per launch
+    attn_avg = statistics.mean(attn_ms)
+    attn_tf = ATTN_FLOP / (attn_avg * 1e-3) / 1e12
+
+    # ---- recache of all layers (sink + window), bulk rewrite
+    ll.ll_kv_recache_write(cache, -1, kn, vn, 0, S + W, stream)
+    torch.cuda.synchronize(dev)
+    r_ms = []
+    for _ in range(max(3, args.steps)):
+        e0.record(stream)
+        ll.ll_kv_recache_write(cache, -1, kn, vn, 0, S + W, stream)
+        e1.record(stream)
+        e1.synchronize()
+        r_ms.append(e0.elapsed_time(e1))
+    rec_ms = statistics.median(r_ms)
+
+    # ---- append alone (HBM-bound)
+    a_ms = []
+    for _ in range(max(3, args.steps)):
+        e0.record(stream)
+        for l in range(L):
+            ll.ll_kv_append(cache, l, ks[l], vs[l], stream)
+        e1.record(stream)
+        e1.synchronize()
+        a_ms.append(e0.elapsed_time(e1) / L)
+    app_ms = statistics.median(a_ms)
+
+    # ---- end to end through the C ABI from pinned host buffers
+    hq = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+    hk = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+    hv = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+    ho = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+    for l in range(L):
+        hq[l].copy_(qs[l].cpu())
+        hk[l].copy_(ks[l].cpu())
+        hv[l].copy_(vs[l].cpu())
+    dq = [torch.empty_like(qs[0]) for _ in range(2)]
+    dk = [torch.empty_like(qs[0]) for _ in range(2)]
+    dv = [torch.empty_like(qs[0]) for _ in range(2)]
+    do = [torch.empty_like(qs[0]) for _ in range(2)]
+    h2d = torch.cuda.Stream(dev)
+    d2h = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event() for _ in range(L)]
+    done = [torch.cuda.Event() for _ in range(L)]
+    freed = [torch.cuda.Event() for _ in range(L)]
+
+    def e2e_step():
+        # layer l's inputs stream in on h2d while layer l-1 computes; outputs stream
+        # out on d2h; two device buffers per tensor
+        # (L is even, so buffer b of layer l was last used by layer (l - 2) mod L,
+        # possibly of the previous step; an event never recorded is a no-op wait)
+        for l in range(L):
+            b = l & 1
+            h2d.wait_event(freed[(l - 2) % L])       # compute done with input buffer b
+            with torch.cuda.stream(h2d):
+                dq[b].copy_(hq[l], non_blocking=True)
+                dk[b].copy_(hk[l], non_blocking=True)
+                dv[b].copy_(hv[l], non_blocking=True)
+                ready[l].record(h2d)
+            stream.wait_event(ready[l])
+            stream.wait_event(done[(l - 2) % L])     # output buffer b drained to host
+            ll.ll_attn_sink_window(dq[b], dk[b], dv[b], cache, l, do[b], stream)
+            ll.ll_kv_append(cache, l, dk[b], dv[b], stream)
+            freed[l].record(stream)
+            d2h.wait_event(freed[l])
+            with torch.cuda.stream(d2h):
+                ho[l].copy_(do[b], non_blocking=True)
+                done[l].record(d2h)
+
+    for _ in range(min(args.warmup, 2)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    _barrier(world)
+    e0.record(stream)
+    h2d.wait_stream(stream)
+    d2h.wait_stream(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    stream.wait_stream(d2h)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    e2e_value = world * ATTN_FLOP * L / (e2e_ms * 1e-3) / 1e12
+
+    # ---- CPU oracle baseline (rank 0, single GPU only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, threads, _ = cpu_oracle_sample()
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+
+    status = ll.ll_debug_status(cache)
+    cache.close()
+    traffic = ATTN_TRAFFIC if (ATTN_TRAFFIC is not None and ATTN_TRAFFIC_SRC_SHA == _kernel_sha()) else None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "wan1.3b-30layer-chunk-step", "layers": L, "heads": H, "head_dim": D,
+                   "tokens_per_frame": T, "frames_per_chunk": F, "sink_frames": S, "window_frames": W,
+                   "visible_keys": NK, "cache": "full (steady state)",
+                   "step": "per layer: ll_attn_sink_window + ll_kv_append",
+                   "l2": "inputs larger than L2: 30-layer cache 3.45 GB + 1.7 GB activations per step",
+                   "parallelism": f"replicas x{world} (independent streams)"},
+        "pct_bf16_peak": value / peak_tf,
+        "latent_frames_per_s": world * F / (ms_step * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": attn_tf / peak_tf, "traffic": traffic, "peak_kind": f"{peak_kind} bf16 burst",
+                     "kernel": "attn_sink_window_kernel<128>", "launch_ms": attn_avg,
+                     "algorithmic_flop_per_launch": ATTN_FLOP, "min_bytes_per_launch": ATTN_MIN_BYTES},
+        "append": {"ms_per_layer": app_ms, "gbs": APPEND_BYTES / (app_ms * 1e-3) / 1e9,
+                   "frac_hbm": APPEND_BYTES / (app_ms * 1e-3) / 1e9 / peak_gbs},
+        "recache": {"ms_all_layers": rec_ms, "bytes": RECACHE_BYTES,
+                    "gbs": RECACHE_BYTES / (rec_ms * 1e-3) / 1e9,
+                    "frac_hbm": RECACHE_BYTES / (rec_ms * 1e-3) / 1e9 / peak_gbs},
+        "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * L * TQ * H * D * 2, "d2h_bytes_per_step": L * TQ * H * D * 2},
+        "gpu_launches": 2 * L * args.steps,
+        "clocks": clk.summary(),
+        "cpu_baseline": cpu,
+        "device_status": status,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = _dist_init(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

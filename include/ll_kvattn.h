@@ -1,0 +1,170 @@
+/*
+ * ll_kvattn.h - C ABI of the LongLive sink + window chunk-attention library
+ * for NVIDIA B200 (sm_100a).
+ *
+ * The library implements the per-layer hot path of frame-level causal
+ * autoregressive video generation with a bounded KV cache:
+ *
+ *   - a KV cache per layer holding the K/V of a permanently kept frame sink and
+ *     of a short sliding window of recent frames (LongLive explainer, dpshk.com,
+ *     sec. 五 "Short Window Attention" and sec. 六 "Frame Sink": KV cache = sink
+ *     frames' KV + recent window's KV);
+ *   - the append/evict step after each generated chunk (same sections; the
+ *     techwalker.com LONGLIVE article, sec. 六, clears old cache entries
+ *     progressively);
+ *   - the bulk rewrite of the held K/V after a prompt switch, "KV-recache"
+ *     (dpshk.com sec. 三.3 and 三.5; techwalker.com sec. 六);
+ *   - attention of the current chunk's queries over sink + window + the chunk's
+ *     own K/V, full inside the chunk and causal across chunks (LongLive-2.0
+ *     explainer, wmrh.cn, sec. 6).
+ *
+ * Conventions shared by every call
+ *   Notation: L layers, H heads, D head_dim, T tokens per latent frame,
+ *   F frames per chunk, S sink frames, W window frames, Tq = F*T.
+ *   Activation tensors (q, k_cur, v_cur, out, k_new, v_new) are caller-owned
+ *   DEVICE pointers to contiguous bf16 (IEEE bfloat16 bit patterns), token-major
+ *   [tokens][H][D], batch 1, 16-byte aligned. The library never frees them.
+ *   The cache owns all of its device memory from create to destroy; no call
+ *   between those allocates device memory (constant footprint).
+ *   Every call that takes a stream only enqueues work on it; none synchronises
+ *   the host. Calls touching the same layer must be ordered by the caller, on
+ *   one stream or with events. The host-side frame counter of a layer advances
+ *   when ll_kv_append is called (enqueue order = logical order).
+ *   Errors are returned, never raised or aborted; on an error nothing was
+ *   enqueued unless the status is LL_ERR_CUDA (a launch failed), and the cache
+ *   handle stays valid.
+ *   `stream` is a cudaStream_t (NULL = legacy default stream); it is declared
+ *   through the CUDA runtime's own opaque struct so that this header needs no
+ *   CUDA include.
+ *
+ * Window reading: W counts cached frames of EARLIER chunks; the own chunk is
+ * always added on top. A frame below S is a sink frame only; the window holds
+ * the last W non-sink frames before the current chunk.
+ */
+#ifndef LL_KVATTN_H
+#define LL_KVATTN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define LL_API __attribute__((visibility("default")))
+#else
+#define LL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ll_stream_t;     /* == cudaStream_t */
+typedef struct ll_kv_cache ll_kv_cache;      /* opaque; owns the cache memory */
+
+typedef enum {
+  LL_KV_BF16 = 0,       /* K/V stored as bf16 */
+  LL_KV_FP8_E4M3 = 1,   /* E4M3 codes + one fp32 scale per (token, head) row */
+  LL_KV_NVFP4 = 2       /* E2M1 codes, 16-value blocks along D, E4M3 block scale */
+} ll_kv_dtype;
+
+typedef enum {
+  LL_OK = 0,
+  LL_ERR_INVALID_ARG = 1,   /* a range, null, alignment or state check failed */
+  LL_ERR_OOM = 2,           /* device allocation failed at create */
+  LL_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed */
+  LL_ERR_UNSUPPORTED = 4,   /* valid request this build does not implement */
+  LL_ERR_TIMEOUT = 5        /* a bounded in-kernel wait gave up (see ll_debug_status) */
+} ll_status;
+
+/* ll_kv_cache_create - allocate the cache of `layers` layers.
+ *   Layout (device, one allocation): for each layer l and each of K (0), V (1):
+ *   [H][(S+W)*T][D] elements; slots 0..S-1 (frame granularity) hold the sink
+ *   frames, slots S..S+W-1 form a frame-granular ring holding the window.
+ *   Quantised formats add a scale array per layer and K/V:
+ *   FP8 [H][(S+W)*T] fp32; NVFP4 [H][(S+W)*T][D/16] E4M3 bytes.
+ *   The memory is zero-filled at create; frame counters start at 0.
+ *   Supported: layers, heads, tokens_per_frame, frames_per_chunk >= 1;
+ *   head_dim in {64, 128}; sink_frames >= 0, window_frames >= 0,
+ *   sink_frames + window_frames >= 1; (S+W)*T and F*T < 2^31.
+ *   Returns LL_ERR_INVALID_ARG on a bad parameter or null `out`,
+ *   LL_ERR_OOM if the allocation fails, LL_ERR_CUDA if no device is usable.
+ *   On success *out owns the memory until ll_kv_cache_destroy.           */
+LL_API ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per_frame,
+                             int frames_per_chunk, int sink_frames, int window_frames,
+                             ll_kv_dtype kv_dtype, ll_kv_cache **out);
+
+/* ll_kv_append - store the chunk just generated in layer `layer` and evict.
+ *   k_cur, v_cur: [F*T][H][D] bf16 device pointers (the chunk's K and V).
+ *   Frame f = p..p+F-1 (p = frames appended to this layer so far) goes to slot
+ *   f if f < S; otherwise, if f >= p+F-W, to ring slot S + ((f-S) mod W),
+ *   overwriting (evicting) the oldest window frame; other frames (only when
+ *   W < F) are not stored. Quantised caches quantise here. Then p += F.
+ *   Pages: dpshk.com sec. 五/六; techwalker.com sec. 六.                    */
+LL_API ll_status ll_kv_append(ll_kv_cache *cache, int layer, const void *k_cur, const void *v_cur,
+                       ll_stream_t stream);
+
+/* ll_kv_recache_write - KV-recache: overwrite held frames with new K/V.
+ *   layer: 0..L-1, or -1 for all layers at once.
+ *   k_new, v_new: [L'][num_frames*T][H][D] bf16 device pointers, L' = 1 for a
+ *   single layer or L for all layers; frame i of the source replaces logical
+ *   frame first_frame+i of the held context, whose logical order is: sink
+ *   frames 0..s-1, then window frames oldest to newest (s = min(p,S),
+ *   w = min(W, max(0, p-S))). Requires 0 <= first_frame, num_frames >= 1 and
+ *   first_frame + num_frames <= s + w of every addressed layer.
+ *   Frame counters and the ring position are unchanged.
+ *   Sink + window is the default context (dpshk.com sec. 三.3); first_frame = S,
+ *   num_frames = W gives the window-only variant with the sink unchanged
+ *   (techwalker.com sec. 六).                                                */
+LL_API ll_status ll_kv_recache_write(ll_kv_cache *cache, int layer, const void *k_new, const void *v_new,
+                              int first_frame, int num_frames, ll_stream_t stream);
+
+/* ll_attn_sink_window - attention of the current chunk of layer `layer`.
+ *   q, k_cur, v_cur: [F*T][H][D] bf16 device pointers (the chunk's Q, K, V);
+ *   out: [F*T][H][D] bf16 device pointer, written. out may not alias inputs.
+ *   For each head: out = softmax(q K^T / sqrt(D)) V over the keys of
+ *   cache slots [0, s*T) (sink), [S*T, (S+w)*T) (window; held frames in any
+ *   ring order, softmax is order-free) and the chunk's own k_cur/v_cur
+ *   (all Tq of them, no mask inside the chunk). s, w as for recache, taken
+ *   from the layer's frame counter at call time: call it BEFORE ll_kv_append
+ *   of the same chunk. bf16 operands, fp32 accumulation and softmax, the
+ *   probabilities rounded to bf16 for the PV product, bf16 output.
+ *   Quantised caches are dequantised inside the kernel.
+ *   Pages: dpshk.com sec. 五/六; techwalker.com sec. 四/六; wmrh.cn sec. 6.  */
+LL_API ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cur,
+                              ll_kv_cache *cache, int layer, void *out, ll_stream_t stream);
+
+/* ll_kv_cache_destroy - free all memory of the cache (NULL is a no-op).
+ *   Synchronises the device first so that no enqueued work still uses it.  */
+LL_API ll_status ll_kv_cache_destroy(ll_kv_cache *cache);
+
+/* ---- helpers --------------------------------------------------------- */
+
+/* Static string for a status code. Never NULL.                              */
+LL_API const char *ll_status_string(ll_status status);
+
+/* Frames appended so far to `layer` (p) and the cache's total device bytes
+ * (all layers, data + scales). Either output pointer may be NULL.           */
+LL_API ll_status ll_kv_cache_info(const ll_kv_cache *cache, int layer, long long *frames_seen,
+                           size_t *device_bytes);
+
+/* Number of device allocations the library currently holds (all caches).
+ * Constant between create and destroy: the footprint check of a rollout.   */
+LL_API long long ll_allocation_count(void);
+
+/* Raw bytes of one layer, in the order: K data [H][(S+W)*T][...], V data,
+ * then for quantised formats K scales, V scales (layouts as at create).
+ * host_dst must hold `bytes` == ll_kv_export_bytes(cache); the call copies on
+ * `stream` and synchronises that stream before returning.                  */
+LL_API size_t ll_kv_export_bytes(const ll_kv_cache *cache);
+LL_API ll_status ll_kv_cache_export(const ll_kv_cache *cache, int layer, void *host_dst, size_t bytes,
+                             ll_stream_t stream);
+
+/* Device-side status word of the cache's kernels: 0 = fine; otherwise a
+ * bounded wait inside a kernel gave up (code in the low byte, kernel id in
+ * the next byte). Reading synchronises `stream`; `clear` resets it to 0.
+ * A non-zero word also makes this call return LL_ERR_TIMEOUT.              */
+LL_API ll_status ll_debug_status(ll_kv_cache *cache, unsigned int *word, int clear, ll_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LL_KVATTN_H */

@@ -1,0 +1,178 @@
+"""Python binding of libll_kvattn.so (the C ABI in include/ll_kvattn.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels. torch is used for device memory and streams; tensors passed in
+must be CUDA, bf16, contiguous, 16-byte aligned, token-major [tokens][H][D].
+Raw integer device pointers are accepted too.
+
+Importing this module loads the in-tree library and fails loudly if it is
+missing (build it with `python -m kv_cache_attention_ll_b200.build`); there is
+no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libll_kvattn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build the CUDA library first "
+                      "(python -m kv_cache_attention_ll_b200.build); there is no fallback")
+_lib = ctypes.CDLL(LIB_PATH)
+
+LL_KV_BF16, LL_KV_FP8_E4M3, LL_KV_NVFP4 = 0, 1, 2
+LL_OK, LL_ERR_INVALID_ARG, LL_ERR_OOM, LL_ERR_CUDA, LL_ERR_UNSUPPORTED, LL_ERR_TIMEOUT = range(6)
+_DTYPES = {"bf16": LL_KV_BF16, "fp8": LL_KV_FP8_E4M3, "nvfp4": LL_KV_NVFP4}
+
+_vp, _i, _ll, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+_sig = {
+    "ll_kv_cache_create": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
+    "ll_kv_append": (_i, [_vp, _i, _vp, _vp, _vp]),
+    "ll_kv_recache_write": (_i, [_vp, _i, _vp, _vp, _i, _i, _vp]),
+    "ll_attn_sink_window": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _vp]),
+    "ll_kv_cache_destroy": (_i, [_vp]),
+    "ll_status_string": (ctypes.c_char_p, [_i]),
+    "ll_kv_cache_info": (_i, [_vp, _i, ctypes.POINTER(_ll), ctypes.POINTER(_sz)]),
+    "ll_allocation_count": (_ll, []),
+    "ll_kv_export_bytes": (_sz, [_vp]),
+    "ll_kv_cache_export": (_i, [_vp, _i, _vp, _sz, _vp]),
+    "ll_debug_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint), _i, _vp]),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+class LLError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {ll_status_string(status)} ({status})")
+
+
+def ll_status_string(status: int) -> str:
+    return _lib.ll_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != LL_OK:
+        raise LLError(status, where)
+
+
+def _ptr(x) -> int:
+    if x is None:
+        return 0
+    if isinstance(x, int):
+        return x
+    import torch
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"expected a torch tensor or an int pointer, got {type(x)}")
+    if not x.is_cuda or x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise ValueError("tensors must be CUDA, bfloat16 and contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class KVCache:
+    """Owner of one ll_kv_cache handle (the device memory lives in the library)."""
+
+    def __init__(self, handle: int, layers, heads, head_dim, tokens_per_frame, frames_per_chunk,
+                 sink_frames, window_frames, kv_dtype):
+        self.handle = handle
+        self.layers, self.heads, self.head_dim = layers, heads, head_dim
+        self.tokens_per_frame, self.frames_per_chunk = tokens_per_frame, frames_per_chunk
+        self.sink_frames, self.window_frames, self.kv_dtype = sink_frames, window_frames, kv_dtype
+
+    @property
+    def tq(self) -> int:
+        return self.frames_per_chunk * self.tokens_per_frame
+
+    def close(self):
+        if self.handle:
+            h, self.handle = self.handle, 0
+            _check(_lib.ll_kv_cache_destroy(h), "ll_kv_cache_destroy")
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+
+def ll_kv_cache_create(layers: int, heads: int, head_dim: int, tokens_per_frame: int, frames_per_chunk: int,
+                       sink_frames: int, window_frames: int, kv_dtype="bf16") -> KVCache:
+    dt = _DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    h = _vp()
+    _check(_lib.ll_kv_cache_create(layers, heads, head_dim, tokens_per_frame, frames_per_chunk, sink_frames,
+                                   window_frames, dt, ctypes.byref(h)), "ll_kv_cache_create")
+    return KVCache(h.value, layers, heads, head_dim, tokens_per_frame, frames_per_chunk, sink_frames,
+                   window_frames, kv_dtype)
+
+
+def ll_kv_append(cache: KVCache, layer: int, k_cur, v_cur, stream=None):
+    _check(_lib.ll_kv_append(cache.handle, layer, _ptr(k_cur), _ptr(v_cur), _stream(stream)), "ll_kv_append")
+
+
+def ll_kv_recache_write(cache: KVCache, layer: int, k_new, v_new, first_frame: int, num_frames: int, stream=None):
+    _check(_lib.ll_kv_recache_write(cache.handle, layer, _ptr(k_new), _ptr(v_new), first_frame, num_frames,
+                                    _stream(stream)), "ll_kv_recache_write")
+
+
+def ll_attn_sink_window(q, k_cur, v_cur, cache: KVCache, layer: int, out, stream=None):
+    _check(_lib.ll_attn_sink_window(_ptr(q), _ptr(k_cur), _ptr(v_cur), cache.handle, layer, _ptr(out),
+                                    _stream(stream)), "ll_attn_sink_window")
+
+
+def ll_kv_cache_destroy(cache: KVCache):
+    cache.close()
+
+
+def ll_kv_cache_info(cache: KVCache, layer: int = 0):
+    p, b = _ll(), _sz()
+    _check(_lib.ll_kv_cache_info(cache.handle, layer, ctypes.byref(p), ctypes.byref(b)), "ll_kv_cache_info")
+    return p.value, b.value
+
+
+def ll_allocation_count() -> int:
+    return _lib.ll_allocation_count()
+
+
+def ll_kv_export_bytes(cache: KVCache) -> int:
+    return _lib.ll_kv_export_bytes(cache.handle)
+
+
+def ll_kv_cache_export(cache: KVCache, layer: int, stream=None) -> bytes:
+    n = ll_kv_export_bytes(cache)
+    buf = ctypes.create_string_buffer(n)
+    _check(_lib.ll_kv_cache_export(cache.handle, layer, ctypes.cast(buf, _vp), n, _stream(stream)),
+           "ll_kv_cache_export")
+    return buf.raw
+
+
+def ll_debug_status(cache: KVCache, clear: bool = False, stream=None) -> int:
+    w = ctypes.c_uint()
+    st = _lib.ll_debug_status(cache.handle, ctypes.byref(w), int(clear), _stream(stream))
+    if st not in (LL_OK, LL_ERR_TIMEOUT):
+        _check(st, "ll_debug_status")
+    return w.value
+
+
+def raw_lib():
+    """The loaded ctypes library (for tests that call the C ABI directly)."""
+    return _lib

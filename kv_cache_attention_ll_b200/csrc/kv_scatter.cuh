@@ -1,0 +1,184 @@
+// kv_scatter.cuh - append/evict and KV-recache writes into the ring cache.
+//
+// Both operations copy whole frames of token-major K/V ([tokens][H][D] bf16, as
+// a QKV projection emits them) into the head-major cache planes
+// ([plane][slots][D], plane = (layer*2 + kv)*H + head), frame f of the source
+// landing in frame slot `slot_of(f)`:
+//   append  (LongLive explainer, dpshk.com, sec. 五/六: sink kept, oldest window
+//            frame evicted): f < S -> f; f >= p+F-W -> S + ((f-S) mod W); else skip
+//   recache (dpshk.com sec. 三.5; techwalker.com LONGLIVE article sec. 六): logical
+//            frame k of the held context -> k if k < s, else the ring slot of
+//            absolute frame p - w + (k - s).
+// One thread moves one 16-byte vector (8 values) of K and the same vector of V;
+// the D/8 threads of one (token, head) row are consecutive lanes, so reads are
+// fully coalesced and each row is written as one contiguous 128/256-byte run.
+// Quantising formats reduce the row (FP8) or the 16-value block (NVFP4) with
+// lane shuffles inside that group and write codes + scales.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+namespace llk {
+
+enum ScatterMode : int { SCATTER_APPEND = 0, SCATTER_RECACHE = 1 };
+enum CacheFormat : int { FMT_BF16 = 0, FMT_FP8 = 1, FMT_NVFP4 = 2 };
+
+struct ScatterParams {
+  const uint4 *src_k;        // [n_layers][n_frames*T][H][D] bf16
+  const uint4 *src_v;
+  uint8_t *data;             // cache data base (all layers)
+  uint8_t *scales;           // cache scale base (quantised formats) or null
+  long long total_vec;       // n_layers * n_frames*T * H * (D/8)
+  int H, D, T, slots;        // slots = (S+W)*T per plane
+  int layer0;                // first destination layer
+  int n_frames;              // frames per source layer
+  int mode;                  // ScatterMode
+  int S, W, F;               // cache geometry
+  int p;                     // frames appended before (append) / held state (recache)
+  int s, w, first;           // recache: held sink/window frames, first logical frame
+};
+
+__device__ __forceinline__ int scatter_slot(const ScatterParams &q, int fi) {
+  if (q.mode == SCATTER_APPEND) {
+    const int f = q.p + fi;
+    if (f < q.S) return f;
+    if (q.W > 0 && f >= q.p + q.F - q.W) return q.S + (f - q.S) % q.W;
+    return -1;
+  }
+  const int k = q.first + fi;
+  if (k < q.s) return k;
+  const int a = q.p - q.w + (k - q.s);
+  return q.S + (a - q.S) % q.W;
+}
+
+// 8 fp32 -> 8 E4M3 codes (round to nearest even, saturating), element 0 in byte 0
+__device__ __forceinline__ uint2 e4m3x8(const float (&y)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint16_t h;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(y[2 * i + 1]), "f"(y[2 * i]));
+    w[i] = h;
+  }
+  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
+}
+
+// 8 fp32 -> 8 E2M1 codes packed in 4 bytes, element 2i in the low nibble of byte i
+__device__ __forceinline__ uint32_t e2m1x8(const float (&y)[8]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+  return out;
+}
+
+// one E4M3 code -> its fp32 value (exact)
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+  uint32_t h2;
+  // the code sits in both bytes, so either half of the f16 pair holds its value
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>((code & 0xFF) * 0x101u)));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFF)));
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&x)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) {
+  const int vpr = q.D >> 3;                    // vectors per (token, head) row: 8 or 16
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  // warp-uniform trip count: every lane runs every iteration so that the
+  // row-group shuffles of the quantising formats always see all 32 lanes
+  for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x; base < q.total_vec; base += stride) {
+    const long long i = base + threadIdx.x;
+    const bool in = i < q.total_vec;
+    const long long ic = in ? i : 0;
+    const int vec = static_cast<int>(ic % vpr);
+    const long long row = ic / vpr;                         // (layer_i, token, head)
+    const int hh = static_cast<int>(row % q.H);
+    const long long lt = row / q.H;                         // (layer_i, token)
+    const int li = static_cast<int>(lt / (static_cast<long long>(q.n_frames) * q.T));
+    const int tok = static_cast<int>(lt % (static_cast<long long>(q.n_frames) * q.T));
+    const int fi = tok / q.T, t = tok % q.T;
+    const int slot = scatter_slot(q, fi);
+    const bool act = in && slot >= 0;
+    const int layer = q.layer0 + li;
+    const long long plane_k = (static_cast<long long>(layer) * 2 + 0) * q.H + hh;
+    const long long plane_v = plane_k + q.H;
+    const long long drow = static_cast<long long>(slot) * q.T + t;   // row inside a plane
+    uint4 vk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    if (act) {
+      vk = __ldg(q.src_k + ic);
+      vv = __ldg(q.src_v + ic);
+    }
+    if constexpr (FMT == FMT_BF16) {
+      if (act) {
+        uint4 *dk = reinterpret_cast<uint4 *>(q.data) + (plane_k * q.slots + drow) * vpr + vec;
+        uint4 *dv = reinterpret_cast<uint4 *>(q.data) + (plane_v * q.slots + drow) * vpr + vec;
+        *dk = vk;
+        *dv = vv;
+      }
+    } else if constexpr (FMT == FMT_FP8) {
+      // per (token, head) row: scale = amax/448 (1 if amax == 0), codes = E4M3(x * (1/scale))
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        float x[8];
+        bf16x8_to_f32(kv == 0 ? vk : vv, x);
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+        for (int o = 1; o < vpr; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        const float scale = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+        const float inv = __fdiv_rn(1.0f, scale);
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(x[e], inv);
+        const uint2 codes = e4m3x8(y);
+        if (act) {
+          const long long plane = kv == 0 ? plane_k : plane_v;
+          uint2 *dc = reinterpret_cast<uint2 *>(q.data + (plane * q.slots + drow) * q.D) + vec;
+          *dc = codes;
+          if (vec == 0) reinterpret_cast<float *>(q.scales)[plane * q.slots + drow] = scale;
+        }
+      }
+    } else {
+      // NVFP4: per 16-value block (two lanes): sb = E4M3(amax/6); codes = E2M1(x / sb), 0 if sb == 0
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        float x[8];
+        bf16x8_to_f32(kv == 0 ? vk : vv, x);
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        float sv[8] = {__fdiv_rn(amax, 6.0f), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        const uint32_t sb_code = e4m3x8(sv).x & 0xFFu;
+        const float sb = e4m3_to_f32(sb_code);
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = sb == 0.f ? 0.f : __fdiv_rn(x[e], sb);
+        const uint32_t codes = sb == 0.f ? 0u : e2m1x8(y);
+        if (act) {
+          const long long plane = kv == 0 ? plane_k : plane_v;
+          uint32_t *dc = reinterpret_cast<uint32_t *>(q.data + (plane * q.slots + drow) * (q.D / 2)) + vec;
+          *dc = codes;
+          if ((vec & 1) == 0) q.scales[(plane * q.slots + drow) * (q.D / 16) + (vec >> 1)] = static_cast<uint8_t>(sb_code);
+        }
+      }
+    }
+  }
+}
+
+}  // namespace llk

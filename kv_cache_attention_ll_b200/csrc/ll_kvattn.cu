@@ -1,0 +1,358 @@
+// ll_kvattn.cu - host side of the C ABI declared in include/ll_kvattn.h:
+// the cache object (one device allocation per cache, zero-filled, never grown),
+// argument validation, ring-buffer bookkeeping (host-side frame counters),
+// TMA descriptor setup and the kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "ll_kvattn.h"
+#include "attn_sink_window.cuh"
+#include "kv_scatter.cuh"
+
+struct ll_kv_cache {
+  int L, H, D, T, F, S, W;
+  ll_kv_dtype dtype;
+  int device;
+  long long slots;            // (S+W)*T rows per plane
+  uint8_t *base;              // the one allocation
+  size_t bytes;               // its size
+  uint8_t *data;              // [L][2][H][slots][row bytes]
+  uint8_t *scales;            // quantised formats: [L][2][H][slots][...]
+  unsigned *err;              // device status word
+  size_t data_plane_bytes;    // bytes of one plane's data
+  size_t scale_plane_bytes;   // bytes of one plane's scales
+  std::vector<long long> p;   // frames appended per layer
+  CUtensorMap tm_cache;       // bf16 cache planes (D, slots, L*2*H)
+};
+
+namespace {
+
+std::atomic<long long> g_alloc_count{0};
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D bf16 tensor map: dims (d0 innermost, d1, d2), strides of d1 and d2 in bytes,
+// box (b0, b1, b2), 128-byte swizzle, zero fill outside the tensor.
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
+                 uint64_t s2_bytes, uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// token-major activation [Tq][H][D] viewed as (D, H, Tq), box (64, 1, 128)
+bool make_act_map(CUtensorMap *m, const void *p, int Tq, int H, int D) {
+  return make_map_3d(m, p, D, H, Tq, static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(H) * D * 2, 64, 1, 128);
+}
+
+void held(const ll_kv_cache *c, int layer, int *s, int *w) {
+  const long long p = c->p[layer];
+  *s = static_cast<int>(p < c->S ? p : c->S);
+  long long ww = p - c->S;
+  if (ww < 0) ww = 0;
+  if (ww > c->W) ww = c->W;
+  *w = static_cast<int>(ww);
+}
+
+// The frame counter as the kernels see it: only whether p < S and the ring
+// position (p - S) mod W matter once p >= S + W, so very long rollouts are
+// folded into int range without changing any slot.
+int kernel_p(const ll_kv_cache *c, int layer) {
+  const long long p = c->p[layer];
+  if (p <= (1ll << 30)) return static_cast<int>(p);
+  if (c->W == 0) return c->S + c->W;
+  return c->S + c->W + static_cast<int>((p - c->S) % c->W);
+}
+
+int num_sms(int device) {
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
+  return n > 0 ? n : 148;
+}
+
+template <int D>
+ll_status launch_attn(const llk::AttnParams &prm, int grid, cudaStream_t stream) {
+  using C = llk::AttnCfg<D>;
+  static std::atomic<unsigned> configured_mask{0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned bit = 1u << (dev & 31);
+  if (!(configured_mask.load() & bit)) {
+    if (cudaFuncSetAttribute(llk::attn_sink_window_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_ALLOC) != cudaSuccess)
+      return LL_ERR_CUDA;
+    configured_mask.fetch_or(bit);
+  }
+  llk::attn_sink_window_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, cudaStream_t stream) {
+  if (q.total_vec == 0) return LL_OK;
+  long long blocks = (q.total_vec + 255) / 256;
+  const long long cap = static_cast<long long>(num_sms(c->device)) * 8;
+  if (blocks > cap) blocks = cap;
+  switch (c->dtype) {
+    case LL_KV_BF16: llk::kv_scatter_kernel<llk::FMT_BF16><<<static_cast<int>(blocks), 256, 0, stream>>>(q); break;
+    case LL_KV_FP8_E4M3: llk::kv_scatter_kernel<llk::FMT_FP8><<<static_cast<int>(blocks), 256, 0, stream>>>(q); break;
+    case LL_KV_NVFP4: llk::kv_scatter_kernel<llk::FMT_NVFP4><<<static_cast<int>(blocks), 256, 0, stream>>>(q); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+llk::ScatterParams scatter_base(const ll_kv_cache *c, const void *k, const void *v) {
+  llk::ScatterParams q;
+  std::memset(&q, 0, sizeof(q));
+  q.src_k = static_cast<const uint4 *>(k);
+  q.src_v = static_cast<const uint4 *>(v);
+  q.data = c->data;
+  q.scales = c->scales;
+  q.H = c->H;
+  q.D = c->D;
+  q.T = c->T;
+  q.slots = static_cast<int>(c->slots);
+  q.S = c->S;
+  q.W = c->W;
+  q.F = c->F;
+  return q;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ll_status_string(ll_status s) {
+  switch (s) {
+    case LL_OK: return "ok";
+    case LL_ERR_INVALID_ARG: return "invalid argument";
+    case LL_ERR_OOM: return "out of device memory";
+    case LL_ERR_CUDA: return "CUDA error";
+    case LL_ERR_UNSUPPORTED: return "unsupported";
+    case LL_ERR_TIMEOUT: return "in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+long long ll_allocation_count(void) { return g_alloc_count.load(); }
+
+ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per_frame, int frames_per_chunk,
+                             int sink_frames, int window_frames, ll_kv_dtype kv_dtype, ll_kv_cache **out) {
+  if (!out) return LL_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (layers < 1 || heads < 1 || tokens_per_frame < 1 || frames_per_chunk < 1) return LL_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LL_ERR_INVALID_ARG;
+  if (sink_frames < 0 || window_frames < 0 || sink_frames + window_frames < 1) return LL_ERR_INVALID_ARG;
+  if (kv_dtype != LL_KV_BF16 && kv_dtype != LL_KV_FP8_E4M3 && kv_dtype != LL_KV_NVFP4) return LL_ERR_INVALID_ARG;
+  const long long slots = static_cast<long long>(sink_frames + window_frames) * tokens_per_frame;
+  const long long tq = static_cast<long long>(frames_per_chunk) * tokens_per_frame;
+  if (slots >= (1ll << 31) || tq >= (1ll << 31)) return LL_ERR_INVALID_ARG;
+  const long long planes = static_cast<long long>(layers) * 2 * heads;
+  if (planes >= (1ll << 31)) return LL_ERR_INVALID_ARG;
+
+  size_t row_bytes = 0, scale_row_bytes = 0;
+  switch (kv_dtype) {
+    case LL_KV_BF16: row_bytes = head_dim * 2; break;
+    case LL_KV_FP8_E4M3: row_bytes = head_dim; scale_row_bytes = 4; break;
+    case LL_KV_NVFP4: row_bytes = head_dim / 2; scale_row_bytes = head_dim / 16; break;
+  }
+  const size_t data_plane = static_cast<size_t>(slots) * row_bytes;
+  const size_t scale_plane = static_cast<size_t>(slots) * scale_row_bytes;
+  const size_t data_bytes = data_plane * planes;
+  const size_t scale_off = (data_bytes + 255) & ~size_t(255);
+  const size_t scale_bytes = scale_plane * planes;
+  const size_t err_off = (scale_off + scale_bytes + 255) & ~size_t(255);
+  const size_t total = err_off + 256;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
+  ll_kv_cache *c = new (std::nothrow) ll_kv_cache();
+  if (!c) return LL_ERR_OOM;
+  c->L = layers; c->H = heads; c->D = head_dim; c->T = tokens_per_frame; c->F = frames_per_chunk;
+  c->S = sink_frames; c->W = window_frames; c->dtype = kv_dtype; c->device = dev; c->slots = slots;
+  c->p.assign(layers, 0);
+  c->data_plane_bytes = data_plane;
+  c->scale_plane_bytes = scale_plane;
+  void *mem = nullptr;
+  cudaError_t e = cudaMalloc(&mem, total);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    delete c;
+    return e == cudaErrorMemoryAllocation ? LL_ERR_OOM : LL_ERR_CUDA;
+  }
+  g_alloc_count.fetch_add(1);
+  c->base = static_cast<uint8_t *>(mem);
+  c->bytes = total;
+  c->data = c->base;
+  c->scales = scale_bytes ? c->base + scale_off : nullptr;
+  c->err = reinterpret_cast<unsigned *>(c->base + err_off);
+  if (cudaMemset(mem, 0, total) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(mem);
+    g_alloc_count.fetch_sub(1);
+    delete c;
+    return LL_ERR_CUDA;
+  }
+  std::memset(&c->tm_cache, 0, sizeof(c->tm_cache));
+  if (kv_dtype == LL_KV_BF16) {
+    if (!make_map_3d(&c->tm_cache, c->data, head_dim, slots, planes, static_cast<uint64_t>(head_dim) * 2,
+                     static_cast<uint64_t>(slots) * head_dim * 2, 64, 128, 1)) {
+      cudaFree(mem);
+      g_alloc_count.fetch_sub(1);
+      delete c;
+      return LL_ERR_CUDA;
+    }
+  }
+  *out = c;
+  return LL_OK;
+}
+
+ll_status ll_kv_cache_destroy(ll_kv_cache *c) {
+  if (!c) return LL_OK;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(c->device);
+  cudaDeviceSynchronize();
+  const cudaError_t e = cudaFree(c->base);
+  g_alloc_count.fetch_sub(1);
+  cudaSetDevice(prev);
+  delete c;
+  return e == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+ll_status ll_kv_cache_info(const ll_kv_cache *c, int layer, long long *frames_seen, size_t *device_bytes) {
+  if (!c || layer < 0 || layer >= c->L) return LL_ERR_INVALID_ARG;
+  if (frames_seen) *frames_seen = c->p[layer];
+  if (device_bytes) *device_bytes = c->bytes;
+  return LL_OK;
+}
+
+size_t ll_kv_export_bytes(const ll_kv_cache *c) {
+  if (!c) return 0;
+  return 2 * (c->data_plane_bytes + c->scale_plane_bytes) * static_cast<size_t>(c->H);
+}
+
+ll_status ll_kv_cache_export(const ll_kv_cache *c, int layer, void *host_dst, size_t bytes, ll_stream_t stream) {
+  if (!c || !host_dst || layer < 0 || layer >= c->L || bytes != ll_kv_export_bytes(c)) return LL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *dst = static_cast<uint8_t *>(host_dst);
+  const size_t dlayer = 2 * c->data_plane_bytes * c->H;
+  if (cudaMemcpyAsync(dst, c->data + dlayer * layer, dlayer, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return LL_ERR_CUDA;
+  if (c->scales) {
+    const size_t slayer = 2 * c->scale_plane_bytes * c->H;
+    if (cudaMemcpyAsync(dst + dlayer, c->scales + slayer * layer, slayer, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      return LL_ERR_CUDA;
+  }
+  return cudaStreamSynchronize(s) == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+ll_status ll_debug_status(ll_kv_cache *c, unsigned int *word, int clear, ll_stream_t stream) {
+  if (!c || !word) return LL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned w = 0;
+  if (cudaMemcpyAsync(&w, c->err, sizeof(w), cudaMemcpyDeviceToHost, s) != cudaSuccess) return LL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LL_ERR_CUDA;
+  if (clear && cudaMemsetAsync(c->err, 0, sizeof(unsigned), s) != cudaSuccess) return LL_ERR_CUDA;
+  *word = w;
+  return w ? LL_ERR_TIMEOUT : LL_OK;
+}
+
+ll_status ll_kv_append(ll_kv_cache *c, int layer, const void *k_cur, const void *v_cur, ll_stream_t stream) {
+  if (!c || layer < 0 || layer >= c->L || !k_cur || !v_cur || !aligned16(k_cur) || !aligned16(v_cur))
+    return LL_ERR_INVALID_ARG;
+  llk::ScatterParams q = scatter_base(c, k_cur, v_cur);
+  q.mode = llk::SCATTER_APPEND;
+  q.layer0 = layer;
+  q.n_frames = c->F;
+  q.p = kernel_p(c, layer);
+  q.total_vec = static_cast<long long>(c->F) * c->T * c->H * (c->D / 8);
+  const ll_status st = launch_scatter(c, q, reinterpret_cast<cudaStream_t>(stream));
+  if (st == LL_OK) c->p[layer] += c->F;
+  return st;
+}
+
+ll_status ll_kv_recache_write(ll_kv_cache *c, int layer, const void *k_new, const void *v_new, int first_frame,
+                              int num_frames, ll_stream_t stream) {
+  if (!c || layer < -1 || layer >= c->L || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))
+    return LL_ERR_INVALID_ARG;
+  if (first_frame < 0 || num_frames < 1) return LL_ERR_INVALID_ARG;
+  const int l0 = layer < 0 ? 0 : layer;
+  const int nl = layer < 0 ? c->L : 1;
+  // every addressed layer must hold the same context (same counter) so that one
+  // launch can apply one logical->slot map
+  int s = 0, w = 0;
+  held(c, l0, &s, &w);
+  for (int l = l0; l < l0 + nl; ++l) {
+    if (c->p[l] != c->p[l0]) return LL_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(first_frame) + num_frames > s + w) return LL_ERR_INVALID_ARG;
+  llk::ScatterParams q = scatter_base(c, k_new, v_new);
+  q.mode = llk::SCATTER_RECACHE;
+  q.layer0 = l0;
+  q.n_frames = num_frames;
+  q.p = kernel_p(c, l0);
+  q.s = s;
+  q.w = w;
+  q.first = first_frame;
+  q.total_vec = static_cast<long long>(nl) * num_frames * c->T * c->H * (c->D / 8);
+  return launch_scatter(c, q, reinterpret_cast<cudaStream_t>(stream));
+}
+
+ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cur, ll_kv_cache *c, int layer,
+                              void *out, ll_stream_t stream) {
+  if (!c || layer < 0 || layer >= c->L || !q || !k_cur || !v_cur || !out) return LL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out)) return LL_ERR_INVALID_ARG;
+  if (out == q || out == k_cur || out == v_cur) return LL_ERR_INVALID_ARG;
+  if (c->dtype != LL_KV_BF16) return LL_ERR_UNSUPPORTED;
+  const int Tq = c->F * c->T;
+  int s = 0, w = 0;
+  held(c, layer, &s, &w);
+  llk::AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!make_act_map(&prm.tm_q, q, Tq, c->H, c->D) || !make_act_map(&prm.tm_kcur, k_cur, Tq, c->H, c->D) ||
+      !make_act_map(&prm.tm_vcur, v_cur, Tq, c->H, c->D))
+    return LL_ERR_CUDA;
+  prm.tm_cache = c->tm_cache;
+  prm.out = static_cast<__nv_bfloat16 *>(out);
+  prm.err = c->err;
+  prm.H = c->H;
+  prm.Tq = Tq;
+  prm.n_cache = (s + w) * c->T;
+  prm.plane_k = (layer * 2 + 0) * c->H;
+  prm.plane_v = (layer * 2 + 1) * c->H;
+  prm.num_q_tiles = (Tq + 127) / 128;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->D)));
+  const int grid = prm.num_q_tiles * c->H;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+"""CPU checks of the boundary: the library loads, exports every symbol that
+include/ll_kvattn.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ll_kvattn.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"LL_API\s+[\w\s\*]+?\b(ll_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("ll_kv_cache_create", "ll_kv_append", "ll_kv_recache_write", "ll_attn_sink_window",
+              "ll_kv_cache_destroy"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import kv_cache_attention_ll_b200 as ll
+    lib = ctypes.CDLL(ll.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    import kv_cache_attention_ll_b200 as ll
+    assert ll.ll_status_string(ll.LL_OK) == "ok"
+    assert ll.ll_status_string(ll.LL_ERR_TIMEOUT).startswith("in-kernel")
+    assert ll.ll_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("args", [
+    (0, 2, 64, 16, 3, 3, 6, 0),      # no layers
+    (1, 0, 64, 16, 3, 3, 6, 0),      # no heads
+    (1, 2, 96, 16, 3, 3, 6, 0),      # unsupported head_dim
+    (1, 2, 64, 0, 3, 3, 6, 0),       # no tokens per frame
+    (1, 2, 64, 16, 0, 3, 6, 0),      # no frames per chunk
+    (1, 2, 64, 16, 3, -1, 6, 0),     # negative sink
+    (1, 2, 64, 16, 3, 0, 0, 0),      # neither sink nor window
+    (1, 2, 64, 16, 3, 3, 6, 7),      # unknown dtype
+    (1, 2, 64, 1 << 30, 3, 3, 6, 0),  # too many slots
+])
+def test_create_rejects_bad_arguments_before_cuda(args):
+    import kv_cache_attention_ll_b200 as ll
+    lib = ll.raw_lib()
+    h = ctypes.c_void_p(1234)
+    assert lib.ll_kv_cache_create(*args, ctypes.byref(h)) == ll.LL_ERR_INVALID_ARG
+    assert h.value is None
+
+
+def test_calls_reject_null_cache():
+    import kv_cache_attention_ll_b200 as ll
+    lib = ll.raw_lib()
+    assert lib.ll_kv_append(None, 0, 16, 16, None) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_kv_recache_write(None, -1, 16, 16, 0, 1, None) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_attn_sink_window(16, 16, 16, None, 0, 32, None) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_kv_cache_destroy(None) == ll.LL_OK
+    assert lib.ll_kv_export_bytes(None) == 0
+    assert lib.ll_allocation_count() == 0
