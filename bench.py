@@ -32,19 +32,23 @@ if ROOT not in sys.path:
 
 METRIC = "sink+window chunk-attention TFLOP/s & % BF16 peak; ms/chunk-step (30 layers)"
 UNIT = "TFLOP/s"
-# Wan-1.3B-shaped stack
+# Wan-1.3B-shaped stack (L is set from --layers; 30 by default)
 L, H, D, T, F, S, W = 30, 12, 128, 1560, 3, 3, 9
 TQ = F * T
 NK = (S + W + F) * T                       # visible keys in steady state: 23400
 ATTN_FLOP = 4.0 * TQ * NK * D * H          # per layer: QK^T and PV over visible keys only
 APPEND_BYTES = 2 * 2 * TQ * H * D * 2      # K and V, read + write
-RECACHE_BYTES = 2 * 2 * L * (S + W) * T * H * D * 2
+
+
+def recache_bytes(layers: int) -> int:
+    return 2 * 2 * layers * (S + W) * T * H * D * 2
+
 ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out + cached K, V
 # ncu DRAM traffic of one attention launch at this shape and the kernel sources it
 # was taken with (profiles/attn_sink_window_wan1.3b.md); reported only while the
 # kernel is unchanged.
-ATTN_TRAFFIC = None
-ATTN_TRAFFIC_SRC_SHA = None
+ATTN_TRAFFIC = 168.34e6        # mean of the two captured launches (167.0 MB, 169.7 MB)
+ATTN_TRAFFIC_SRC_SHA = "07c2efa4b0cbe297"
 
 
 def _peaks():
@@ -77,7 +81,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -129,11 +133,13 @@ def _dist_init(args):
 
 
 def _max_over_ranks(x: float, world: int) -> float:
+    """MAX of a per-rank time over all ranks (the slowest replica sets the pace)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -144,39 +150,52 @@ def _barrier(world):
         dist.barrier()
 
 
-def cpu_oracle_sample(seconds_target: float = 12.0):
+_ORACLE_INPUTS = None
+
+
+def _oracle_inputs():
+    """Seeded bf16 history of one layer up to chunk 4 (p = 12 = S + W: the cache is full)."""
+    global _ORACLE_INPUTS
+    if _ORACLE_INPUTS is None:
+        import numpy as np
+        from seeded_inputs import chunk_qkv
+        c = 4
+        hk, hv = [], []
+        for cc in range(c + 1):
+            q, k, v = chunk_qkv(1, 0, cc, TQ, H, D)
+            hk.append(k)
+            hv.append(v)
+        _ORACLE_INPUTS = (c, q, np.concatenate(hk), np.concatenate(hv))
+    return _ORACLE_INPUTS
+
+
+def cpu_oracle_sample(seconds_target: float = 12.0, n_rows: int | None = None):
     """Times the CPU oracle on a bounded sample of the workload: sampled query
     rows of one steady-state layer-chunk (all 12 heads, all 23400 visible keys).
-    Returns (TFLOP/s, sample description, threads, seconds)."""
+    Returns (TFLOP/s, sample description, threads, rows used)."""
     import numpy as np
     import oracle
-    from seeded_inputs import chunk_qkv
-    c = 4                                    # p = 12 = S + W: the cache is full
-    hk, hv = [], []
-    for cc in range(c + 1):
-        q, k, v = chunk_qkv(1, 0, cc, TQ, H, D)
-        hk.append(k)
-        hv.append(v)
-    kh, vh = np.concatenate(hk), np.concatenate(hv)
+    c, q, kh, vh = _oracle_inputs()
     rng = np.random.default_rng(5)
-    rows = np.sort(rng.choice(TQ, 16, replace=False))
+    if n_rows is None:
+        rows = np.sort(rng.choice(TQ, 16, replace=False))
+        t0 = time.perf_counter()
+        oracle.sink_window_attention(q, kh, vh, c, S, W, F, T, rows=rows)
+        dt = time.perf_counter() - t0
+        n_rows = int(max(16, min(TQ, 16 * seconds_target / max(dt, 1e-3))))
+    rows = np.sort(rng.choice(TQ, n_rows, replace=False))
     t0 = time.perf_counter()
     oracle.sink_window_attention(q, kh, vh, c, S, W, F, T, rows=rows)
     dt = time.perf_counter() - t0
-    n = int(max(16, min(TQ, 16 * seconds_target / max(dt, 1e-3))))
-    rows = np.sort(rng.choice(TQ, n, replace=False))
-    t0 = time.perf_counter()
-    oracle.sink_window_attention(q, kh, vh, c, S, W, F, T, rows=rows)
-    dt = time.perf_counter() - t0
-    flop = 4.0 * n * NK * D * H
+    flop = 4.0 * n_rows * NK * D * H
     try:
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
         threads = os.cpu_count() or 1
-    desc = (f"fp64 numpy oracle, {n} of {TQ} query rows x {H} heads of one steady-state layer-chunk "
+    desc = (f"fp64 numpy oracle, {n_rows} of {TQ} query rows x {H} heads of one steady-state layer-chunk "
             f"({NK} visible keys), {dt:.1f} s")
-    return flop / dt / 1e12, desc, threads, dt
+    return flop / dt / 1e12, desc, threads, n_rows
 
 
 def run_reference(args, world, rank):
@@ -184,8 +203,10 @@ def run_reference(args, world, rank):
         return
     vals = []
     desc = threads = None
+    n_rows = None
+    per_step = max(0.5, args.ref_budget_s / (args.warmup + args.steps))
     for i in range(args.warmup + args.steps):
-        v, desc, threads, _ = cpu_oracle_sample(seconds_target=max(2.0, 60.0 / (args.warmup + args.steps)))
+        v, desc, threads, n_rows = cpu_oracle_sample(seconds_target=per_step, n_rows=n_rows)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.mean(vals)
@@ -246,16 +267,14 @@ def run_ours(args, world, rank, local):
                 ev[l][1].record(stream)
             ll.ll_kv_append(cache, l, ks[l], vs[l], stream)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    _barrier(world)
-
-    # ---- device-timed steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # clocks are sampled from the start of the warm-up to the end of the timed steps
     with ClockSampler(local) as clk:
+        for _ in range(args.warmup):
+            step()
         torch.cuda.synchronize(dev)
         _barrier(world)
+        # ---- device-timed steps
         e0.record(stream)
         for i in range(args.steps):
             step(attn_ev[i])
@@ -296,61 +315,70 @@ def run_ours(args, world, rank, local):
     app_ms = statistics.median(a_ms)
 
     # ---- end to end through the C ABI from pinned host buffers
-    hq = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
-    hk = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
-    hv = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
-    ho = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
-    for l in range(L):
-        hq[l].copy_(qs[l].cpu())
-        hk[l].copy_(ks[l].cpu())
-        hv[l].copy_(vs[l].cpu())
-    dq = [torch.empty_like(qs[0]) for _ in range(2)]
-    dk = [torch.empty_like(qs[0]) for _ in range(2)]
-    dv = [torch.empty_like(qs[0]) for _ in range(2)]
-    do = [torch.empty_like(qs[0]) for _ in range(2)]
-    h2d = torch.cuda.Stream(dev)
-    d2h = torch.cuda.Stream(dev)
-    ready = [torch.cuda.Event() for _ in range(L)]
-    done = [torch.cuda.Event() for _ in range(L)]
-    freed = [torch.cuda.Event() for _ in range(L)]
-
-    def e2e_step():
-        # layer l's inputs stream in on h2d while layer l-1 computes; outputs stream
-        # out on d2h; two device buffers per tensor
-        # (L is even, so buffer b of layer l was last used by layer (l - 2) mod L,
-        # possibly of the previous step; an event never recorded is a no-op wait)
+    def run_e2e():
+        hq = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+        hk = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+        hv = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
+        ho = [torch.empty(TQ, H, D, dtype=torch.bfloat16).pin_memory() for _ in range(L)]
         for l in range(L):
-            b = l & 1
-            h2d.wait_event(freed[(l - 2) % L])       # compute done with input buffer b
-            with torch.cuda.stream(h2d):
-                dq[b].copy_(hq[l], non_blocking=True)
-                dk[b].copy_(hk[l], non_blocking=True)
-                dv[b].copy_(hv[l], non_blocking=True)
-                ready[l].record(h2d)
-            stream.wait_event(ready[l])
-            stream.wait_event(done[(l - 2) % L])     # output buffer b drained to host
-            ll.ll_attn_sink_window(dq[b], dk[b], dv[b], cache, l, do[b], stream)
-            ll.ll_kv_append(cache, l, dk[b], dv[b], stream)
-            freed[l].record(stream)
-            d2h.wait_event(freed[l])
-            with torch.cuda.stream(d2h):
-                ho[l].copy_(do[b], non_blocking=True)
-                done[l].record(d2h)
+            hq[l].copy_(qs[l].cpu())
+            hk[l].copy_(ks[l].cpu())
+            hv[l].copy_(vs[l].cpu())
+        dq = [torch.empty_like(qs[0]) for _ in range(2)]
+        dk = [torch.empty_like(qs[0]) for _ in range(2)]
+        dv = [torch.empty_like(qs[0]) for _ in range(2)]
+        do = [torch.empty_like(qs[0]) for _ in range(2)]
+        h2d = torch.cuda.Stream(dev)
+        d2h = torch.cuda.Stream(dev)
+        ready = [torch.cuda.Event() for _ in range(2)]
+        done = [torch.cuda.Event() for _ in range(2)]     # D2H of buffer b finished
+        freed = [torch.cuda.Event() for _ in range(2)]    # compute finished with buffer b
 
-    for _ in range(min(args.warmup, 2)):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    _barrier(world)
-    e0.record(stream)
-    h2d.wait_stream(stream)
-    d2h.wait_stream(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    stream.wait_stream(d2h)
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-    e2e_value = world * ATTN_FLOP * L / (e2e_ms * 1e-3) / 1e12
+        def e2e_step():
+            # layer l's inputs stream in on h2d while the previous layer computes;
+            # outputs stream out on d2h; two device buffers per tensor, alternating.
+            # Waiting on an event waits for its latest record, i.e. the previous use
+            # of that buffer (a never-recorded event is a no-op wait).
+            for l in range(L):
+                b = l & 1
+                h2d.wait_event(freed[b])
+                with torch.cuda.stream(h2d):
+                    dq[b].copy_(hq[l], non_blocking=True)
+                    dk[b].copy_(hk[l], non_blocking=True)
+                    dv[b].copy_(hv[l], non_blocking=True)
+                    ready[b].record(h2d)
+                stream.wait_event(ready[b])
+                stream.wait_event(done[b])
+                ll.ll_attn_sink_window(dq[b], dk[b], dv[b], cache, l, do[b], stream)
+                ll.ll_kv_append(cache, l, dk[b], dv[b], stream)
+                freed[b].record(stream)
+                d2h.wait_event(freed[b])
+                with torch.cuda.stream(d2h):
+                    ho[l].copy_(do[b], non_blocking=True)
+                    done[b].record(d2h)
+
+        for _ in range(min(args.warmup, 2)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        _barrier(world)
+        e0.record(stream)
+        h2d.wait_stream(stream)
+        d2h.wait_stream(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        stream.wait_stream(d2h)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        e2e_value = world * ATTN_FLOP * L / (e2e_ms * 1e-3) / 1e12
+
+        return e2e_ms, e2e_value
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, e2e_value = run_e2e()
+        e2e = {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": 3 * L * TQ * H * D * 2, "d2h_bytes_per_step": L * TQ * H * D * 2}
 
     # ---- CPU oracle baseline (rank 0, single GPU only)
     cpu = None
@@ -379,11 +407,10 @@ def run_ours(args, world, rank, local):
                      "algorithmic_flop_per_launch": ATTN_FLOP, "min_bytes_per_launch": ATTN_MIN_BYTES},
         "append": {"ms_per_layer": app_ms, "gbs": APPEND_BYTES / (app_ms * 1e-3) / 1e9,
                    "frac_hbm": APPEND_BYTES / (app_ms * 1e-3) / 1e9 / peak_gbs},
-        "recache": {"ms_all_layers": rec_ms, "bytes": RECACHE_BYTES,
-                    "gbs": RECACHE_BYTES / (rec_ms * 1e-3) / 1e9,
-                    "frac_hbm": RECACHE_BYTES / (rec_ms * 1e-3) / 1e9 / peak_gbs},
-        "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
-                "h2d_bytes_per_step": 3 * L * TQ * H * D * 2, "d2h_bytes_per_step": L * TQ * H * D * 2},
+        "recache": {"ms_all_layers": rec_ms, "bytes": recache_bytes(L),
+                    "gbs": recache_bytes(L) / (rec_ms * 1e-3) / 1e9,
+                    "frac_hbm": recache_bytes(L) / (rec_ms * 1e-3) / 1e9 / peak_gbs},
+        "e2e": e2e,
         "gpu_launches": 2 * L * args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
@@ -396,11 +423,17 @@ def run_ours(args, world, rank, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--layers", type=int, default=30, help="stack depth (30 = the Wan-1.3B stack)")
+    ap.add_argument("--ref-budget-s", type=float, default=90.0,
+                    help="CPU seconds the reference arm spends in total (bounded sample per step)")
     args = ap.parse_args()
+    global L
+    L = args.layers
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = _dist_init(args)
