@@ -17,11 +17,12 @@
 // and sums in the epilogue. Tiles past the valid keys are never visited; only
 // the last tile of each segment masks its tail columns.
 //
-// Roles (320 threads):
+// Roles (384 threads, three warpgroups):
 //   warps 0-3  softmax warpgroup 0 (thread t owns query row t = TMEM lane t)
 //   warps 4-7  softmax warpgroup 1
 //   warp 8     TMA producer (Q once, then K and V tiles into an NST-deep ring)
-//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 9     TMEM allocator and tcgen05.mma issuer
+//   warps 10-11 idle (they complete the third warpgroup for register reallocation)
 //
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D). P_g (bf16) overwrites the first 64 columns of S_g and is
@@ -76,7 +77,11 @@ struct AttnCfg {
   static constexpr int OFF_STATS = OFF_Q;
   static constexpr int SMEM_BYTES = OFF_MISC + 32;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;      // slack for 1024-byte alignment
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;   // 3 warpgroups; warps 10-11 idle
+  // registers: launched with 384 x 168 = 64512; the producer/MMA warpgroup drops
+  // to 64 and the softmax warpgroups rise to 216: 128*64 + 256*216 = 63488 <= 64512
+  static constexpr uint32_t REGS_SOFTMAX = 216;
+  static constexpr uint32_t REGS_ISSUE = 64;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, D, 0, 1);
@@ -84,13 +89,19 @@ struct AttnCfg {
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
 };
 
+// Which pairs of probabilities (bit e%8 for pair e) take exp2 on the FMA pipe
+// instead of MUFU. MUFU runs 4 lanes per clock per sub-partition, so one softmax
+// warp alone needs 1024 clocks for 128 exp2 per row; moving a share of them to
+// FMA-pipe polynomials balances the two pipes.
+constexpr unsigned kPolyPairs = 0x88u;
+
 __device__ __forceinline__ int tile_valid(int j, int nc, int n_cache, int Tq) {
   if (j < nc) return min(128, n_cache - j * 128);
   return min(128, Tq - (j - nc) * 128);
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1) attn_sink_window_kernel(const __grid_constant__ AttnParams prm) {
+__global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_constant__ AttnParams prm) {
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -156,19 +167,27 @@ __global__ void __launch_bounds__(320, 1) attn_sink_window_kernel(const __grid_c
 #define TM_S(g) (tmem + 128u * static_cast<uint32_t>(g))
 #define TM_O(g) (tmem + 256u + static_cast<uint32_t>(D) * static_cast<uint32_t>(g))
 
+  if (warp >= 8) {
+  // each role sets its register budget inside its own branch, so that the
+  // allocation limit is unambiguous at every point of the role's code
+  regs_dec<C::REGS_ISSUE>();
   if (warp == 8) {
     // ------------------------------------------------------------- producer
-    if (lane == 0) {
-      uint8_t *sq = smem + C::OFF_Q;
+    // The whole warp runs this loop converged; one elected lane issues.
+    uint8_t *sq = smem + C::OFF_Q;
+    if (elect_one()) {
       mbar_arrive_expect_tx(q_full, C::Q_BYTES);
       for (int b = 0; b < C::NBOX; ++b) tma_load_3d(sq + b * C::BOX_BYTES, &prm.tm_q, q_full, b * 64, h, q0);
-      int issued_k = 0, issued_v = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int st = j % C::NST;
-        const uint32_t par = ((j / C::NST) & 1) ^ 1;
-        uint8_t *sk = smem + C::OFF_K + st * C::TILE_BYTES;
-        uint8_t *sv = smem + C::OFF_V + st * C::TILE_BYTES;
-        if (!mbar_wait(k_empty + st, par, abort_flag, prm.err, KID_ATTN)) break;
+    }
+    __syncwarp();
+    int issued_k = 0, issued_v = 0;
+    for (int j = 0; j < n_tiles; ++j) {
+      const int st = j % C::NST;
+      const uint32_t par = ((j / C::NST) & 1) ^ 1;
+      uint8_t *sk = smem + C::OFF_K + st * C::TILE_BYTES;
+      uint8_t *sv = smem + C::OFF_V + st * C::TILE_BYTES;
+      if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, par, abort_flag, prm.err, KID_ATTN))) break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(k_full + st, C::TILE_BYTES);
         if (j < nc) {
           for (int b = 0; b < C::NBOX; ++b)
@@ -177,8 +196,11 @@ __global__ void __launch_bounds__(320, 1) attn_sink_window_kernel(const __grid_c
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_3d(sk + b * C::BOX_BYTES, &prm.tm_kcur, k_full + st, b * 64, h, (j - nc) * C::BN);
         }
-        issued_k = j + 1;
-        if (!mbar_wait(v_empty + st, par, abort_flag, prm.err, KID_ATTN)) break;
+      }
+      __syncwarp();
+      issued_k = j + 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, par, abort_flag, prm.err, KID_ATTN))) break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(v_full + st, C::TILE_BYTES);
         if (j < nc) {
           for (int b = 0; b < C::NBOX; ++b)
@@ -187,69 +209,93 @@ __global__ void __launch_bounds__(320, 1) attn_sink_window_kernel(const __grid_c
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_3d(sv + b * C::BOX_BYTES, &prm.tm_vcur, v_full + st, b * 64, h, (j - nc) * C::BN);
         }
-        issued_v = j + 1;
       }
-      if (*abort_flag) {
-        mbar_wait_drain(q_full, 0);
-        // every load issued must land before the CTA exits: wait for the last
-        // NST of each kind (earlier ones were consumed, so they have landed)
-        for (int j = issued_k > C::NST ? issued_k - C::NST : 0; j < issued_k; ++j)
-          mbar_wait_drain(k_full + j % C::NST, (j / C::NST) & 1);
-        for (int j = issued_v > C::NST ? issued_v - C::NST : 0; j < issued_v; ++j)
-          mbar_wait_drain(v_full + j % C::NST, (j / C::NST) & 1);
-      }
+      __syncwarp();
+      issued_v = j + 1;
     }
+    if (*abort_flag && lane == 0) {
+      mbar_wait_drain(q_full, 0);
+      // every load issued must land before the CTA exits: wait for the last
+      // NST of each kind (earlier ones were consumed, so they have landed)
+      for (int j = issued_k > C::NST ? issued_k - C::NST : 0; j < issued_k; ++j)
+        mbar_wait_drain(k_full + j % C::NST, (j / C::NST) & 1);
+      for (int j = issued_v > C::NST ? issued_v - C::NST : 0; j < issued_v; ++j)
+        mbar_wait_drain(v_full + j % C::NST, (j / C::NST) & 1);
+    }
+    __syncwarp();
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(q_full, 0, abort_flag, prm.err, KID_ATTN);
-      const uint32_t sq = smem_u32(smem + C::OFF_Q);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j % C::NST;
-        if (!mbar_wait(k_full + st, (j / C::NST) & 1, abort_flag, prm.err, KID_ATTN)) return false;
-        tc_fence_after();
-        const uint32_t sk = smem_u32(smem + C::OFF_K + st * C::TILE_BYTES);
+    // The whole warp runs this loop converged (operands stay warp-uniform);
+    // one elected lane issues each tcgen05 instruction.
+    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, abort_flag, prm.err, KID_ATTN));
+    // Shared-memory descriptors are built once; each MMA only adds a constant
+    // to the start-address field (bits 0-13, address >> 4). Every operand lies
+    // below 256 KB of shared memory, so the field never carries into LBO.
+    const uint64_t dq0 = smem_desc(smem_u32(smem + C::OFF_Q), 16, 1024, 2);
+    const uint64_t dk0 = smem_desc(smem_u32(smem + C::OFF_K), 16, 1024, 2);
+    const uint64_t dv0 = smem_desc(smem_u32(smem + C::OFF_V), C::BOX_BYTES, 1024, 2);
+    auto issue_s = [&](int j) -> bool {
+      const int st = j % C::NST;
+      if (!__all_sync(0xffffffffu, mbar_wait(k_full + st, (j / C::NST) & 1, abort_flag, prm.err, KID_ATTN)))
+        return false;
+      tc_fence_after();
+      const uint64_t dk = dk0 + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
+      const uint32_t d_tmem = TM_S(j & 1);
+      // one elected block issues the whole group (an elect per MMA costs more
+      // than the MMA itself); operands were computed by the converged warp
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-          const uint64_t da = smem_desc(sq + off, 16, 1024, 2);
-          const uint64_t db = smem_desc(sk + off, 16, 1024, 2);
-          mma_bf16_ss(TM_S(j & 1), da, db, C::IDESC_S, kk > 0 ? 1u : 0u);
+          // K step kk: box kk/4 (64 head-dim columns each), 32-byte slice kk%4 of the 128-byte row
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::BOX_BYTES + (kk & 3) * 32) >> 4);
+          mma_bf16_ss(d_tmem, dq0 + off, dk + off, C::IDESC_S, kk > 0 ? 1u : 0u);
         }
         mma_commit(k_empty + st);
         mma_commit(s_full + (j & 1));
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && n_tiles > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int g = j & 1, it = j >> 1, st = j % C::NST;
-        if (!mbar_wait(p_full + g, it & 1, abort_flag, prm.err, KID_ATTN)) break;
-        if (!mbar_wait(v_full + st, (j / C::NST) & 1, abort_flag, prm.err, KID_ATTN)) break;
-        tc_fence_after();
-        const uint32_t sv = smem_u32(smem + C::OFF_V + st * C::TILE_BYTES);
+      }
+      __syncwarp();
+      return true;
+    };
+    if (ok) ok = issue_s(0);
+    if (ok && n_tiles > 1) ok = issue_s(1);
+    for (int j = 0; ok && j < n_tiles; ++j) {
+      const int g = j & 1, it = j >> 1, st = j % C::NST;
+      if (!__all_sync(0xffffffffu, mbar_wait(p_full + g, it & 1, abort_flag, prm.err, KID_ATTN))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(v_full + st, (j / C::NST) & 1, abort_flag, prm.err, KID_ATTN))) break;
+      tc_fence_after();
+      const uint64_t dv = dv0 + static_cast<uint64_t>((st * C::TILE_BYTES) >> 4);
+      const uint32_t o_tmem = TM_O(g), p_tmem = TM_S(g);
+      const uint32_t acc0 = it > 0 ? 1u : 0u;
+      if (elect_one()) {
 #pragma unroll
         for (int kk = 0; kk < C::BN / 16; ++kk) {
-          // V tile: rows = keys (K dim of this product), 128-byte rows of 64 head-dim
-          // values, boxes of 64 head-dim columns C::BOX_BYTES apart (MN-major operand)
-          const uint64_t db = smem_desc(sv + kk * 16 * 128, C::BOX_BYTES, 1024, 2);
-          mma_bf16_ts(TM_O(g), TM_S(g) + kk * 8, db, C::IDESC_O, (it > 0 || kk > 0) ? 1u : 0u);
+          // V tile: rows = keys (the K dim of this product), 16 keys = 2048 bytes per
+          // step; boxes of 64 head-dim columns C::BOX_BYTES apart (MN-major operand);
+          // P_g: 16 keys = 8 bf16x2 columns of tensor memory per step
+          mma_bf16_ts(o_tmem, p_tmem + kk * 8, dv + static_cast<uint64_t>((kk * 16 * 128) >> 4), C::IDESC_O,
+                      kk > 0 ? 1u : acc0);
         }
         mma_commit(v_empty + st);
         mma_commit(o_full + g);
-        if (j + 2 < n_tiles) ok = issue_s(j + 2);
       }
-      // every MMA issued must finish before tensor memory is released
+      __syncwarp();
+      if (j + 2 < n_tiles) ok = issue_s(j + 2);
+    }
+    // every MMA issued must finish before tensor memory is released
+    if (elect_one()) {
       mma_commit(mma_done);
       mbar_wait_drain(mma_done, 0);
     }
+    __syncwarp();
+  }
   } else {
+    regs_inc<C::REGS_SOFTMAX>();
     // ------------------------------------------------------- softmax groups
     const int g = warp >> 2;              // warpgroup 0 or 1
     const int row = threadIdx.x & 127;    // TMEM lane == query row in the tile
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float sl2 = prm.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_ref = -INFINITY, l_run = 0.f;
     int it = 0;
     bool ok = true;
     for (int j = g; j < n_tiles; j += 2, ++it) {
@@ -260,60 +306,65 @@ __global__ void __launch_bounds__(320, 1) attn_sink_window_kernel(const __grid_c
         break;
       }
       tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(TM_S(g) + lane_off + c * 32, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r[e]);
-      }
+      // S_g of this tile is complete, and with it every MMA issued before it,
+      // among them the previous PV into O_g: O_g may be rescaled right away, and
+      // no separate wait for that PV is needed (only the last one is awaited).
+      uint32_t sr[128];
+      tmem_ld64(TM_S(g) + lane_off, sr);
+      tmem_ld64(TM_S(g) + lane_off + 64, sr + 64);
       const int valid = tile_valid(j, nc, prm.n_cache, prm.Tq);
       if (valid < 128) {
 #pragma unroll
         for (int e = 0; e < 128; ++e)
-          if (e >= valid) s[e] = -INFINITY;
+          if (e >= valid) sr[e] = __float_as_uint(-INFINITY);
       }
-      float mx = s[0];
+      // row max: four independent chains of 3-input maxima
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int e = 1; e < 128; ++e) mx = fmaxf(mx, s[e]);
-      const float m_tile = mx * sl2;
-      const bool grow = m_tile > m_run + 8.0f;     // lazy rescale: only when the max grows by > 2^8
-      const float m_new = grow ? m_tile : m_run;
-      const float alpha = (grow && it > 0) ? ex2_approx(m_run - m_new) : 1.0f;
-      float sum = 0.f;
+      for (int e = 0; e < 128; e += 8) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pr[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * e], sl2, -m_new));
-          const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * e + 1], sl2, -m_new));
-          sum += p0 + p1;
-          pr[e] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(TM_S(g) + lane_off + c * 32, pr);
+        for (int i = 0; i < 4; ++i)
+          m4[i] = fmax3(m4[i], __uint_as_float(sr[e + 2 * i]), __uint_as_float(sr[e + 2 * i + 1]));
       }
-      l_run = (it > 0 ? l_run * alpha : 0.f) + sum;
-      m_run = m_new;
-      if (it > 0) {
-        // the previous PV of this group must be complete before O is touched
-        if (!__all_sync(0xffffffffu, mbar_wait(o_full + g, (it - 1) & 1, abort_flag, prm.err, KID_ATTN))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+      const float m_tile = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl2;
+      // lazy rescale: the reference max moves only when a tile's max exceeds it
+      // by more than 8 (log2 units), so probabilities stay below 2^8
+      const bool grow = m_tile > m_ref + 8.0f;
+      const float m_new = grow ? m_tile : m_ref;
+      const float alpha = (grow && it > 0) ? ex2_approx(m_ref - m_new) : 1.0f;
+      if (it > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(TM_O(g) + lane_off + c * 32, r);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(TM_O(g) + lane_off + c * 32, r);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(TM_O(g) + lane_off + c * 32, r);
-          }
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(TM_O(g) + lane_off + c * 32, r);
         }
       }
+      // probabilities in pairs: x = s * log2(e)/sqrt(D) - m (packed FMA); pairs
+      // selected by kPolyPairs use the FMA-pipe exp2, the rest MUFU; four packed
+      // partial sums; bf16 pairs written back over S as the A operand of PV
+      const float2 sl2x2 = make_float2(sl2, sl2), nm2 = make_float2(-m_new, -m_new);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      uint32_t pr[64];
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2x2, nm2);
+        float2 pp;
+        if ((kPolyPairs >> (e & 7)) & 1) {
+          pp = exp2_poly2(x);
+        } else {
+          pp.x = ex2_approx(x.x);
+          pp.y = ex2_approx(x.y);
+        }
+        acc[e & 3] = __fadd2_rn(acc[e & 3], pp);
+        pr[e] = pack_bf16x2(pp.x, pp.y);
+      }
+      tmem_st64(TM_S(g) + lane_off, pr);
+      const float2 a03 = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+      l_run = (it > 0 ? l_run * alpha : 0.f) + (a03.x + a03.y);
+      m_ref = m_new;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full + g);
@@ -330,7 +381,7 @@ __global__ void __launch_bounds__(320, 1) attn_sink_window_kernel(const __grid_c
     tc_fence_before();
     named_bar_sync(1, 256);
     if (!*abort_flag) {
-      stat_m[g * 128 + row] = m_run;
+      stat_m[g * 128 + row] = m_ref;
       stat_l[g * 128 + row] = l_run;
       if (row == 0) tile_count[g] = it;
     }

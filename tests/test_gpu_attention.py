@@ -84,3 +84,39 @@ def test_large_logits_rescale_path():
     rescale of O. The softmax is peaked here, so the max-abs bound is the one
     derived from bf16 rounding (see gpu_util.assert_attn_close_derived)."""
     _rollout(21, H=2, D=128, T=64, F=3, S=3, W=6, n_chunks=6, check={2, 5}, qk_scale=4.0)
+
+
+def test_large_max_jump_recompute_path():
+    """The chunk's own keys scaled by 40: its tiles come after the cache tiles and
+    raise the row max by far more than 2^64 over the running reference, which
+    forces the exact recompute of those tiles (and a later O rescale). The
+    softmax is peaked, so the derived bf16 bound applies."""
+    import torch
+    import kv_cache_attention_ll_b200 as ll
+    from gpu_util import to_dev, dev_to_f64, assert_attn_close_derived
+    from seeded_inputs import f32_to_bf16_bits
+    H, D, T, F, S, W = 2, 128, 64, 3, 3, 6
+    Tq = F * T
+    cache = ll.ll_kv_cache_create(1, H, D, T, F, S, W)
+    hk, hv = [], []
+    try:
+        for c in range(5):
+            q = chunk_tensor(KIND_Q, 31, 0, c, Tq, H, D)
+            k = chunk_tensor(KIND_K, 31, 0, c, Tq, H, D)
+            v = chunk_tensor(KIND_V, 31, 0, c, Tq, H, D)
+            if c >= 3:
+                k = f32_to_bf16_bits((bf16_bits_to_f64(k) * 40.0).astype(np.float32))
+            dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+            out = torch.empty_like(dq)
+            ll.ll_attn_sink_window(dq, dk, dv, cache, 0, out)
+            ll.ll_kv_append(cache, 0, dk, dv)
+            hk.append(k)
+            hv.append(v)
+            if c >= 3:
+                torch.cuda.synchronize()
+                ref = oracle.sink_window_attention(q, np.concatenate(hk), np.concatenate(hv), c, S, W, F, T)
+                vmax = float(np.abs(bf16_bits_to_f64(np.concatenate(hv))).max())
+                assert_attn_close_derived(dev_to_f64(out), ref, vmax, f"chunk {c}")
+        assert ll.ll_debug_status(cache) == 0
+    finally:
+        cache.close()
