@@ -380,6 +380,45 @@ def run_ours(args, world, rank, local):
         e2e = {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": 3 * L * TQ * H * D * 2, "d2h_bytes_per_step": L * TQ * H * D * 2}
 
+    # ---- quantised caches: the same stack with K/V stored as FP8 or NVFP4,
+    # quantised on append and dequantised inside the attention kernel
+    quant = {}
+    if not args.no_quant:
+        cache_bytes_bf16 = ll.ll_kv_cache_info(cache, 0)[1]
+        for kvd in ("fp8", "nvfp4"):
+            qc = ll.ll_kv_cache_create(L, H, D, T, F, S, W, kvd)
+            for c in range((S + W + F - 1) // F + 1):
+                for l in range(L):
+                    ll.ll_kv_append(qc, l, ks[l], vs[l], stream)
+            qev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
+                   for _ in range(args.quant_steps)]
+
+            def qstep(ev=None):
+                for l in range(L):
+                    if ev is not None:
+                        ev[l][0].record(stream)
+                    ll.ll_attn_sink_window(qs[l], ks[l], vs[l], qc, l, outs[l], stream)
+                    if ev is not None:
+                        ev[l][1].record(stream)
+                    ll.ll_kv_append(qc, l, ks[l], vs[l], stream)
+
+            for _ in range(3):
+                qstep()
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for i in range(args.quant_steps):
+                qstep(qev[i])
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            q_ms = e0.elapsed_time(e1) / args.quant_steps
+            q_attn = statistics.mean(a.elapsed_time(b) for ev in qev for a, b in ev)
+            qbytes = ll.ll_kv_cache_info(qc, 0)[1]
+            quant[kvd] = {"ms_per_step": q_ms, "value": ATTN_FLOP * L / (q_ms * 1e-3) / 1e12,
+                          "attn_launch_ms": q_attn, "attn_tflops": ATTN_FLOP / (q_attn * 1e-3) / 1e12,
+                          "cache_gb": qbytes / 1e9, "cache_gb_bf16": cache_bytes_bf16 / 1e9,
+                          "device_status": ll.ll_debug_status(qc)}
+            qc.close()
+
     # ---- CPU oracle baseline (rank 0, single GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -414,6 +453,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 2 * L * args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
+        "quantised_cache": quant or None,
         "device_status": status,
     }
     if rank == 0:
@@ -428,6 +468,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-quant", action="store_true", help="skip the FP8 / NVFP4 cache leg")
+    ap.add_argument("--quant-steps", type=int, default=10)
     ap.add_argument("--layers", type=int, default=30, help="stack depth (30 = the Wan-1.3B stack)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="CPU seconds the reference arm spends in total (bounded sample per step)")

@@ -99,21 +99,31 @@ int num_sms(int device) {
   return n > 0 ? n : 148;
 }
 
-template <int D>
+template <int D, int QF>
 ll_status launch_attn(const llk::AttnParams &prm, int grid, cudaStream_t stream) {
-  using C = llk::AttnCfg<D>;
+  using C = llk::AttnCfg<D, QF>;
   static std::atomic<unsigned> configured_mask{0};
   int dev = 0;
   cudaGetDevice(&dev);
   const unsigned bit = 1u << (dev & 31);
   if (!(configured_mask.load() & bit)) {
-    if (cudaFuncSetAttribute(llk::attn_sink_window_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(llk::attn_sink_window_kernel<D, QF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_ALLOC) != cudaSuccess)
       return LL_ERR_CUDA;
     configured_mask.fetch_or(bit);
   }
-  llk::attn_sink_window_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(prm);
+  llk::attn_sink_window_kernel<D, QF><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+template <int D>
+ll_status launch_attn_fmt(ll_kv_dtype dt, const llk::AttnParams &prm, int grid, cudaStream_t stream) {
+  switch (dt) {
+    case LL_KV_BF16: return launch_attn<D, llk::QF_BF16>(prm, grid, stream);
+    case LL_KV_FP8_E4M3: return launch_attn<D, llk::QF_FP8>(prm, grid, stream);
+    case LL_KV_NVFP4: return launch_attn<D, llk::QF_NVFP4>(prm, grid, stream);
+  }
+  return LL_ERR_INVALID_ARG;
 }
 
 ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, cudaStream_t stream) {
@@ -331,7 +341,6 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   if (!c || layer < 0 || layer >= c->L || !q || !k_cur || !v_cur || !out) return LL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out)) return LL_ERR_INVALID_ARG;
   if (out == q || out == k_cur || out == v_cur) return LL_ERR_INVALID_ARG;
-  if (c->dtype != LL_KV_BF16) return LL_ERR_UNSUPPORTED;
   const int Tq = c->F * c->T;
   int s = 0, w = 0;
   held(c, layer, &s, &w);
@@ -350,9 +359,12 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   prm.plane_v = (layer * 2 + 1) * c->H;
   prm.num_q_tiles = (Tq + 127) / 128;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->D)));
+  prm.qdata = c->data;
+  prm.qscales = c->scales;
+  prm.slots = static_cast<int>(c->slots);
   const int grid = prm.num_q_tiles * c->H;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
+  return c->D == 128 ? launch_attn_fmt<128>(c->dtype, prm, grid, st) : launch_attn_fmt<64>(c->dtype, prm, grid, st);
 }
 
 }  // extern "C"

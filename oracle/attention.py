@@ -31,7 +31,12 @@ import numpy as np
 
 
 def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
-    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+    """bf16 bit patterns (uint16) -> exact fp64 values; float arrays pass through
+    (used for caches whose held values are dequantised products)."""
+    a = np.asarray(bits)
+    if np.issubdtype(a.dtype, np.floating):
+        return a.astype(np.float64)
+    return (a.astype(np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
 
 
 def frame_visible(query_frame: int, key_frame: int, S: int, W: int, F: int) -> bool:
@@ -76,8 +81,8 @@ def sink_window_attention(q_bits: np.ndarray, k_hist_bits: np.ndarray, v_hist_bi
     """Attention output of chunk `chunk` in fp64.
 
     q_bits       [F*T][H][D] bf16 bits, the chunk's queries
-    k_hist_bits  [(chunk+1)*F*T][H][D] bf16 bits: K of every frame generated so far,
-                 in generation order, the current chunk's K last (its k_cur)
+    k_hist_bits  [(chunk+1)*F*T][H][D] bf16 bits (or float values): K of every frame
+                 generated so far, in generation order, the current chunk's K last
     v_hist_bits  same for V
     rows         optional subset of query rows (token index in the chunk)
     returns      [len(rows)][H][D] float64

@@ -147,3 +147,25 @@ class CacheModel:
         if not frames:
             return np.zeros((0, self.H) + self.data.shape[4:], dtype=self.data.dtype)
         return np.concatenate(frames, axis=0)
+
+    def held_frames(self, layer: int, kv: int) -> dict:
+        """Held context as {absolute frame number: fp64 values [T][H][D]}: the sink
+        frames 0..s-1 and the window frames p-w..p-1, each dequantised exactly
+        (bf16 bits, or E4M3 code x fp32 row scale, or E2M1 code x E4M3 block
+        scale, in fp64)."""
+        p = self.p[layer]
+        s, w = self.held(layer)
+        out = {}
+        for k in range(s + w):
+            frame = k if k < s else p - w + (k - s)
+            slot = self.logical_slot(layer, k)
+            sl = slice(slot * self.T, (slot + 1) * self.T)
+            if self.kv_dtype == "bf16":
+                rows = (self.data[layer, kv, :, sl].astype(np.uint32) << np.uint32(16)).view(np.float32) \
+                    .astype(np.float64)
+            elif self.kv_dtype == "fp8":
+                rows = quant.fp8_dequantize_rows(self.data[layer, kv, :, sl], self.scales[layer, kv, :, sl])
+            else:
+                rows = quant.nvfp4_dequantize_rows(self.data[layer, kv, :, sl], self.scales[layer, kv, :, sl])
+            out[frame] = np.transpose(rows, (1, 0, 2))
+        return out

@@ -1,0 +1,82 @@
+"""GPU parity of ll_attn_sink_window on FP8 and NVFP4 caches.
+
+The library quantises on append (bit-exact against the oracle, see
+test_gpu_cache.py) and dequantises inside the attention kernel. The oracle
+attends over the exactly dequantised held frames (E4M3 code x fp32 row scale,
+or E2M1 code x E4M3 block scale, in fp64) plus the chunk's own bf16 K/V, with
+its explicit sink + window + block-causal mask.
+
+Bound: the standard max-abs 1e-2 and relative-L2 5e-3. NVFP4 products are exact
+in bf16, so the kernel's error budget is the bf16 one. FP8 products are rounded
+to bf16 once more in the kernel (2.3e-3 relative L2 on its own at the Wan shape),
+which stays inside the same bound."""
+import numpy as np
+import pytest
+
+import oracle
+from seeded_inputs import chunk_qkv, bf16_bits_to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _rollout(kv_dtype, cfg_id, H, D, T, F, S, W, n_chunks, check, rows_per_head=None):
+    import torch
+    import kv_cache_attention_ll_b200 as ll
+    from gpu_util import to_dev, dev_to_f64, assert_attn_close, sample_rows
+    Tq = F * T
+    model = oracle.CacheModel(1, H, D, T, F, S, W, kv_dtype)
+    cache = ll.ll_kv_cache_create(1, H, D, T, F, S, W, kv_dtype)
+    results = []
+    try:
+        for c in range(n_chunks):
+            q, k, v = chunk_qkv(cfg_id, 0, c, Tq, H, D)
+            dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+            out = torch.empty_like(dq)
+            ll.ll_attn_sink_window(dq, dk, dv, cache, 0, out)
+            ll.ll_kv_append(cache, 0, dk, dv)
+            if c in check:
+                # history as the oracle sees it: held frames dequantised, the own
+                # chunk in bf16; frames no longer held are invisible (left zero)
+                n = (c + 1) * Tq
+                kh = np.zeros((n, H, D))
+                vh = np.zeros((n, H, D))
+                for f, vals in model.held_frames(0, 0).items():
+                    kh[f * T:(f + 1) * T] = vals
+                for f, vals in model.held_frames(0, 1).items():
+                    vh[f * T:(f + 1) * T] = vals
+                kh[c * Tq:] = bf16_bits_to_f64(k)
+                vh[c * Tq:] = bf16_bits_to_f64(v)
+                torch.cuda.synchronize()
+                got = dev_to_f64(out)
+                rows = None if rows_per_head is None else sample_rows(Tq, rows_per_head, cfg_id * 77 + c)
+                ref = oracle.sink_window_attention(q, kh, vh, c, S, W, F, T, rows=rows)
+                g = got if rows is None else got[rows]
+                results.append((c, *assert_attn_close(g, ref, f"{kv_dtype} chunk {c}")))
+            model.append(0, k, v)
+        assert ll.ll_debug_status(cache) == 0
+    finally:
+        cache.close()
+    return results
+
+
+@pytest.mark.parametrize("kv_dtype", ["fp8", "nvfp4"])
+def test_quantised_config0_all_chunks(kv_dtype):
+    """Tiny reference geometry (head_dim 64), all 8 chunks."""
+    _rollout(kv_dtype, 40, H=2, D=64, T=16, F=3, S=3, W=6, n_chunks=8, check=set(range(8)))
+
+
+@pytest.mark.parametrize("kv_dtype", ["fp8", "nvfp4"])
+@pytest.mark.parametrize("H,D,T,F,S,W,n", [
+    (3, 128, 50, 3, 2, 5, 7),     # two query tiles, ragged; cache not a multiple of 128
+    (2, 128, 40, 3, 3, 0, 5),     # sink only
+    (1, 64, 129, 1, 2, 3, 7),     # one frame per chunk, one-row tail tile
+])
+def test_quantised_odd_shapes(kv_dtype, H, D, T, F, S, W, n):
+    _rollout(kv_dtype, hash((H, D, T, F, S, W)) & 0xFFF, H, D, T, F, S, W, n, check=set(range(n)))
+
+
+@pytest.mark.parametrize("kv_dtype", ["fp8", "nvfp4"])
+def test_quantised_wan_shape_sampled_rows(kv_dtype):
+    """Wan-1.3B single-layer shape, steady state (chunk 5 holds 12 cached frames)."""
+    res = _rollout(kv_dtype, 41, H=12, D=128, T=1560, F=3, S=3, W=9, n_chunks=6, check={1, 5}, rows_per_head=256)
+    assert len(res) == 2

@@ -111,3 +111,33 @@ def test_constant_footprint_long_rollout():
         m.append(0, k, v)
         assert m.data is buf and m.export_nbytes() == n0
     assert m.held(0) == (3, 9)
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8", "nvfp4"])
+def test_held_frames_are_the_appended_frames_dequantized(kv_dtype):
+    """held_frames maps absolute frame numbers to the values of exactly those
+    frames: bf16 frames bit-exact, quantised frames within the format's error
+    bound of the appended values (and equal to quantising each frame alone)."""
+    from oracle import quant
+    from seeded_inputs import bf16_bits_to_f64
+    S, W, F, T, H, D = 3, 6, 3, 2, 2, 32
+    m = CacheModel(1, H, D, T, F, S, W, kv_dtype)
+    frames = {}
+    for c in range(7):
+        k, v = _chunk(mix_seed(5, 5), c, F, T, H, D)
+        m.append(0, k, v)
+        for fi in range(F):
+            frames[c * F + fi] = k[fi * T:(fi + 1) * T]
+    held = m.held_frames(0, 0)
+    p = 7 * F
+    assert sorted(held) == list(range(S)) + list(range(p - W, p))
+    for f, vals in held.items():
+        x = frames[f]
+        if kv_dtype == "bf16":
+            np.testing.assert_array_equal(vals, bf16_bits_to_f64(x))
+        elif kv_dtype == "fp8":
+            codes, sc = quant.fp8_quantize_rows(np.transpose(x, (1, 0, 2)))
+            np.testing.assert_array_equal(vals, np.transpose(quant.fp8_dequantize_rows(codes, sc), (1, 0, 2)))
+        else:
+            codes, sb = quant.nvfp4_quantize_rows(np.transpose(x, (1, 0, 2)))
+            np.testing.assert_array_equal(vals, np.transpose(quant.nvfp4_dequantize_rows(codes, sb), (1, 0, 2)))
