@@ -79,7 +79,9 @@ typedef enum {
  *   [H][(S+W)*T][D] elements; slots 0..S-1 (frame granularity) hold the sink
  *   frames, slots S..S+W-1 form a frame-granular ring holding the window.
  *   Quantised formats add a scale array per layer and K/V:
- *   FP8 [H][(S+W)*T] fp32; NVFP4 [H][(S+W)*T][D/16] E4M3 bytes.
+ *   FP8 [H][(S+W)*T] fp32; NVFP4 [H][(S+W)*T][D/16] E4M3 bytes; and a bf16
+ *   view of ONE layer's K and V planes (2*H*(S+W)*T*D*2 bytes) that each
+ *   ll_attn_sink_window call refills with the dequantised held frames.
  *   The memory is zero-filled at create; frame counters start at 0.
  *   Supported: layers, heads, tokens_per_frame, frames_per_chunk >= 1;
  *   head_dim in {64, 128}; sink_frames >= 0, window_frames >= 0,
@@ -126,7 +128,11 @@ LL_API ll_status ll_kv_recache_write(ll_kv_cache *cache, int layer, const void *
  *   from the layer's frame counter at call time: call it BEFORE ll_kv_append
  *   of the same chunk. bf16 operands, fp32 accumulation and softmax, the
  *   probabilities rounded to bf16 for the PV product, bf16 output.
- *   Quantised caches are dequantised inside the kernel.
+ *   Quantised caches: the layer's held frames are first dequantised into the
+ *   cache's bf16 view (FP8: E4M3 x row scale rounded to bf16; NVFP4: E2M1 x
+ *   E4M3 block scale, exact in bf16), then attended to like a bf16 cache. The
+ *   view is shared by all layers, so attention calls on one quantised cache
+ *   must be ordered (one stream, or events).
  *   Pages: dpshk.com sec. 五/六; techwalker.com sec. 四/六; wmrh.cn sec. 6.  */
 LL_API ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cur,
                               ll_kv_cache *cache, int layer, void *out, ll_stream_t stream);

@@ -34,7 +34,6 @@
 // order, so P_g is consumed before S_g is overwritten.
 #pragma once
 #include <cuda_bf16.h>
-#include <cuda_fp16.h>
 
 #include "sm100_ptx.cuh"
 
@@ -54,16 +53,9 @@ struct AttnParams {
   int plane_v;           // (l*2 + 1) * H
   int num_q_tiles;
   float scale_log2;      // log2(e) / sqrt(D)
-  // quantised cache formats only (the converter warpgroup reads them directly)
-  const uint8_t *qdata;   // codes [L*2*H][slots][row bytes]
-  const uint8_t *qscales; // FP8: fp32 [L*2*H][slots]; NVFP4: E4M3 [L*2*H][slots][D/16]
-  int slots;              // (S+W)*T rows per plane
 };
 
-// Cache formats of the attention kernel (template parameter QF).
-enum : int { QF_BF16 = 0, QF_FP8 = 1, QF_NVFP4 = 2 };
-
-template <int D, int QF = QF_BF16>
+template <int D>
 struct AttnCfg {
   static constexpr int BM = 128;                    // query rows per CTA
   static constexpr int BN = 128;                    // keys per tile
@@ -71,18 +63,11 @@ struct AttnCfg {
   static constexpr int BOX_BYTES = 128 * 128;       // one box: 128 rows x 128 B
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int TILE_BYTES = BN * D * 2;
-  // K/V ring depth; quantised caches give shared memory to the code staging
-  static constexpr int NST = QF != QF_BF16 ? 2 : (D == 128) ? 3 : 4;
-  // quantised caches: codes of one row of K or V, and the double-buffered
-  // staging area [2][128 rows][K codes | V codes]
-  static constexpr int ROW_CODE_BYTES = QF == QF_FP8 ? D : D / 2;
-  static constexpr int STG_ROW = 2 * ROW_CODE_BYTES;
-  static constexpr int STG_BYTES = QF == QF_BF16 ? 0 : 2 * 128 * STG_ROW;
+  static constexpr int NST = (D == 128) ? 3 : 4;    // K/V ring depth
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NST * TILE_BYTES;
-  static constexpr int OFF_STG = OFF_V + NST * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_STG + STG_BYTES;
+  static constexpr int OFF_BAR = OFF_V + NST * TILE_BYTES;
   // barriers: q_full, k_full[NST], k_empty[NST], v_full[NST], v_empty[NST],
   //           s_full[2], p_full[2], o_full[2], mma_done
   static constexpr int NBAR = 1 + 4 * NST + 7;
@@ -92,15 +77,11 @@ struct AttnCfg {
   static constexpr int OFF_STATS = OFF_Q;
   static constexpr int SMEM_BYTES = OFF_MISC + 32;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;      // slack for 1024-byte alignment
-  // bf16 cache: 3 warpgroups (warps 10-11 idle); quantised caches add a fourth,
-  // the converter warpgroup (warps 12-15)
-  static constexpr int THREADS = QF == QF_BF16 ? 384 : 512;
-  // registers at launch: 384 x 168 = 64512 (bf16) or 512 x 128 = 65536 (quantised).
-  // The softmax warpgroups rise to 216; the other warpgroups drop to 64 (bf16:
-  // 128*64 + 256*216 = 63488 <= 64512) or 40 (quantised: 2*128*40 + 256*216 = 65536)
-  static constexpr uint32_t REGS_SOFTMAX = QF == QF_BF16 ? 216 : 208;
-  static constexpr uint32_t REGS_ISSUE = QF == QF_BF16 ? 64 : 48;
-  static constexpr uint32_t REGS_CONV = 48;
+  static constexpr int THREADS = 384;   // 3 warpgroups; warps 10-11 idle
+  // registers: launched with 384 x 168 = 64512; the producer/MMA warpgroup drops
+  // to 64 and the softmax warpgroups rise to 216: 128*64 + 256*216 = 63488 <= 64512
+  static constexpr uint32_t REGS_SOFTMAX = 216;
+  static constexpr uint32_t REGS_ISSUE = 64;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_S = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16_f32(BM, D, 0, 1);
@@ -119,80 +100,9 @@ __device__ __forceinline__ int tile_valid(int j, int nc, int n_cache, int Tq) {
   return min(128, Tq - (j - nc) * 128);
 }
 
-
-// Dequantisation of quantised cache rows by the converter warpgroup.
-//   FP8   (codes [slots][D], fp32 scale per row): e4m3 -> f16 (exact) -> fp32,
-//         times the row scale, rounded to bf16 (round to nearest even).
-//   NVFP4 (codes [slots][D/2], element 2i in the low nibble; E4M3 scale per 16
-//         values): e2m1 -> f16 and E4M3 -> f16 (both exact), product in f16 (at
-//         most 6 significant bits, inside the f16 range: exact), then bf16 (exact).
-// The output row r of a [128 keys][D] stage tile uses the 128-byte-swizzled
-// layout of the TMA path: head-dim columns d in box d/64, row offset 128 r,
-// 16-byte chunk c at chunk position c ^ (r % 8).
-__device__ __forceinline__ uint32_t f16x2_from_e4m3x2(uint32_t two_codes) {
-  uint32_t d;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(static_cast<uint16_t>(two_codes)));
-  return d;
-}
-__device__ __forceinline__ uint32_t f16x2_from_e2m1x2(uint32_t byte) {
-  uint32_t d;
-  asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(d) : "r"(byte));
-  return d;
-}
-__device__ __forceinline__ uint32_t bf16x2_from_f16x2(uint32_t h2) {
-  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h2));
-  return pack_bf16x2(f.x, f.y);
-}
-
-// 16 bytes of codes -> bf16 values written to `row` (a stage tile row) starting
-// at head-dim column d0. `sc` holds the row scale (FP8) or, for NVFP4, the two
-// E4M3 block scales of these 32 values in its low two bytes.
-template <int QF>
-__device__ __forceinline__ void dequant16(uint4 cv, uint32_t sc, int d0, uint8_t *row, int sw) {
-  auto put = [&](int d, uint4 v) {   // 8 bf16 values of head-dim columns d .. d+7
-    *reinterpret_cast<uint4 *>(row + (d >> 6) * (128 * 128) + ((((d & 63) >> 3) ^ sw) << 4)) = v;
-  };
-  const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
-  if constexpr (QF == QF_FP8) {
-    const float scale = __uint_as_float(sc);
-    const float2 sc2 = make_float2(scale, scale);
-    uint32_t o[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const uint32_t h2 = f16x2_from_e4m3x2(w[i] >> (16 * k));
-        const float2 f = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2 *>(&h2)), sc2);
-        o[2 * i + k] = pack_bf16x2(f.x, f.y);
-      }
-    }
-    put(d0, make_uint4(o[0], o[1], o[2], o[3]));
-    put(d0 + 8, make_uint4(o[4], o[5], o[6], o[7]));
-  } else {
-#pragma unroll
-    for (int blk = 0; blk < 2; ++blk) {
-      const uint32_t s2 = f16x2_from_e4m3x2(((sc >> (8 * blk)) & 0xFFu) * 0x101u);   // scale in both halves
-      uint32_t o[8];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t h2 = f16x2_from_e2m1x2((w[2 * blk + i] >> (8 * k)) & 0xFFu);
-          const __half2 prod =
-              __hmul2(*reinterpret_cast<const __half2 *>(&h2), *reinterpret_cast<const __half2 *>(&s2));
-          o[4 * i + k] = bf16x2_from_f16x2(*reinterpret_cast<const uint32_t *>(&prod));
-        }
-      }
-      put(d0 + 16 * blk, make_uint4(o[0], o[1], o[2], o[3]));
-      put(d0 + 16 * blk + 8, make_uint4(o[4], o[5], o[6], o[7]));
-    }
-  }
-}
-
-template <int D, int QF>
-__global__ void __launch_bounds__(QF == QF_BF16 ? 384 : 512, 1)
-    attn_sink_window_kernel(const __grid_constant__ AttnParams prm) {
-  using C = AttnCfg<D, QF>;
+template <int D>
+__global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_constant__ AttnParams prm) {
+  using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
@@ -247,7 +157,7 @@ __global__ void __launch_bounds__(QF == QF_BF16 ? 384 : 512, 1)
     prefetch_tensormap(&prm.tm_q);
     prefetch_tensormap(&prm.tm_kcur);
     prefetch_tensormap(&prm.tm_vcur);
-    if (QF == QF_BF16) prefetch_tensormap(&prm.tm_cache);
+    prefetch_tensormap(&prm.tm_cache);
   }
   tc_fence_before();
   __syncthreads();
@@ -260,10 +170,7 @@ __global__ void __launch_bounds__(QF == QF_BF16 ? 384 : 512, 1)
   if (warp >= 8) {
   // each role sets its register budget inside its own branch, so that the
   // allocation limit is unambiguous at every point of the role's code
-  if (QF != QF_BF16 && warp >= 12)
-    regs_dec<C::REGS_CONV>();
-  else
-    regs_dec<C::REGS_ISSUE>();
+  regs_dec<C::REGS_ISSUE>();
   if (warp == 8) {
     // ------------------------------------------------------------- producer
     // The whole warp runs this loop converged; one elected lane issues.
@@ -273,12 +180,8 @@ __global__ void __launch_bounds__(QF == QF_BF16 ? 384 : 512, 1)
       for (int b = 0; b < C::NBOX; ++b) tma_load_3d(sq + b * C::BOX_BYTES, &prm.tm_q, q_full, b * 64, h, q0);
     }
     __syncwarp();
-    // quantised caches: every K/V tile comes from the converter warpgroup (it
-    // is the single producer of the ring, so the empty-barrier phases it waits
-    // on are never skipped); this warp then only loads Q
-    const int j0 = QF == QF_BF16 ? 0 : n_tiles;
-    int issued_k = j0, issued_v = j0;
-    for (int j = j0; j < n_tiles; ++j) {
+    int issued_k = 0, issued_v = 0;
+    for (int j = 0; j < n_tiles; ++j) {
       const int st = j % C::NST;
       const uint32_t par = ((j / C::NST) & 1) ^ 1;
       uint8_t *sk = smem + C::OFF_K + st * C::TILE_BYTES;
@@ -286,7 +189,7 @@ __global__ void __launch_bounds__(QF == QF_BF16 ? 384 : 512, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(k_empty + st, par, abort_flag, prm.err, KID_ATTN))) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(k_full + st, C::TILE_BYTES);
-        if (QF == QF_BF16 && j < nc) {
+        if (j < nc) {
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_3d(sk + b * C::BOX_BYTES, &prm.tm_cache, k_full + st, b * 64, j * C::BN, prm.plane_k + h);
         } else {
@@ -299,7 +202,7 @@ __global__ void __launch_bounds__(QF == QF_BF16 ? 384 : 512, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(v_empty + st, par, abort_flag, prm.err, KID_ATTN))) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(v_full + st, C::TILE_BYTES);
-        if (QF == QF_BF16 && j < nc) {
+        if (j < nc) {
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_3d(sv + b * C::BOX_BYTES, &prm.tm_cache, v_full + st, b * 64, j * C::BN, prm.plane_v + h);
         } else {
@@ -314,9 +217,9 @@ __global__ void __launch_bounds__(QF == QF_BF16 ? 384 : 512, 1)
       mbar_wait_drain(q_full, 0);
       // every load issued must land before the CTA exits: wait for the last
       // NST of each kind (earlier ones were consumed, so they have landed)
-      for (int j = max(j0, issued_k - C::NST); j < issued_k; ++j)
+      for (int j = issued_k > C::NST ? issued_k - C::NST : 0; j < issued_k; ++j)
         mbar_wait_drain(k_full + j % C::NST, (j / C::NST) & 1);
-      for (int j = max(j0, issued_v - C::NST); j < issued_v; ++j)
+      for (int j = issued_v > C::NST ? issued_v - C::NST : 0; j < issued_v; ++j)
         mbar_wait_drain(v_full + j % C::NST, (j / C::NST) & 1);
     }
     __syncwarp();
@@ -384,128 +287,6 @@ __global__ void __launch_bounds__(QF == QF_BF16 ? 384 : 512, 1)
       mbar_wait_drain(mma_done, 0);
     }
     __syncwarp();
-  } else if (QF != QF_BF16 && warp >= 12) {
-    // ----------------------------------------------------------- converters
-    // Thread r of this warpgroup handles row r (key slot 128 j + r) of the K and
-    // V tiles of every cache tile j. The codes of tile j+1 are copied with
-    // cp.async into the other staging buffer (and the scales read into
-    // registers) while tile j is dequantised into the stage buffers; the writes
-    // are then made visible to the tensor core (async proxy) and one thread
-    // announces the stage. Like the softmax warps, the loop always runs to
-    // completion so that the warpgroup's named barrier stays matched after an
-    // abort. Shared-memory accesses rotate the 16-byte chunk order by row so
-    // that the 8 rows of a quarter-warp hit 8 different bank groups.
-    constexpr int RB = C::ROW_CODE_BYTES;         // code bytes of one K or V row
-    constexpr int NCH = RB / 16;                  // 16-byte chunks per row
-    const int r = threadIdx.x - 384;
-    const int sw = r & 7;
-    const size_t row_k0 = static_cast<size_t>(prm.plane_k + h) * prm.slots;
-    const size_t row_v0 = static_cast<size_t>(prm.plane_v + h) * prm.slots;
-    uint8_t *stg = smem + C::OFF_STG;
-    // scale words of one row: FP8 the fp32 row scale; NVFP4 D/16 E4M3 bytes
-    constexpr int NSW = QF == QF_FP8 ? 1 : D / 64;   // 32-bit scale words per row
-    auto fetch = [&](int j, uint32_t (&sk)[NSW], uint32_t (&sv)[NSW]) {
-      const int slot = j * C::BN + r;
-      if (slot < prm.n_cache) {
-        const uint8_t *gk = prm.qdata + (row_k0 + slot) * RB;
-        const uint8_t *gv = prm.qdata + (row_v0 + slot) * RB;
-        uint8_t *dst = stg + (j & 1) * (128 * C::STG_ROW) + r * C::STG_ROW;
-#pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-          const int cc = (c + sw) % NCH;
-          cp_async16(dst + cc * 16, gk + cc * 16);
-          cp_async16(dst + RB + cc * 16, gv + cc * 16);
-        }
-        if constexpr (QF == QF_FP8) {
-          sk[0] = __ldg(reinterpret_cast<const uint32_t *>(prm.qscales) + row_k0 + slot);
-          sv[0] = __ldg(reinterpret_cast<const uint32_t *>(prm.qscales) + row_v0 + slot);
-        } else {
-#pragma unroll
-          for (int i = 0; i < NSW; ++i) {
-            sk[i] = __ldg(reinterpret_cast<const uint32_t *>(prm.qscales + (row_k0 + slot) * (D / 16)) + i);
-            sv[i] = __ldg(reinterpret_cast<const uint32_t *>(prm.qscales + (row_v0 + slot) * (D / 16)) + i);
-          }
-        }
-      }
-      cp_async_commit();
-    };
-    uint32_t sk[NSW], sv[NSW], nk[NSW], nv[NSW];
-    if (nc > 0) fetch(0, sk, sv);
-    int tma_issued = nc;   // own-chunk tiles are loaded by TMA from thread 0
-    for (int j = 0; j < n_tiles; ++j) {
-      const int st = j % C::NST;
-      const uint32_t par = ((j / C::NST) & 1) ^ 1;
-      if (j < nc) {
-        if (j + 1 < nc) {
-          fetch(j + 1, nk, nv);
-          cp_async_wait<1>();       // the copies of tile j have landed
-        } else {
-          cp_async_wait<0>();
-        }
-      }
-      mbar_wait(k_empty + st, par, abort_flag, prm.err, KID_ATTN);
-      mbar_wait(v_empty + st, par, abort_flag, prm.err, KID_ATTN);
-      __syncwarp();
-      uint8_t *sk_stage = smem + C::OFF_K + st * C::TILE_BYTES;
-      uint8_t *sv_stage = smem + C::OFF_V + st * C::TILE_BYTES;
-      if (j >= nc) {
-        // the chunk's own K/V (bf16): TMA, completion counted on the full barriers
-        if (r == 0 && !*abort_flag) {
-          mbar_arrive_expect_tx(k_full + st, C::TILE_BYTES);
-          for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d(sk_stage + b * C::BOX_BYTES, &prm.tm_kcur, k_full + st, b * 64, h, (j - nc) * C::BN);
-          mbar_arrive_expect_tx(v_full + st, C::TILE_BYTES);
-          for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d(sv_stage + b * C::BOX_BYTES, &prm.tm_vcur, v_full + st, b * 64, h, (j - nc) * C::BN);
-          tma_issued = j + 1;
-        }
-        continue;
-      }
-      uint8_t *rk = sk_stage + r * 128;
-      uint8_t *rv = sv_stage + r * 128;
-      if (j * C::BN + r < prm.n_cache) {
-        const uint8_t *src = stg + (j & 1) * (128 * C::STG_ROW) + r * C::STG_ROW;
-#pragma unroll 2
-        for (int c = 0; c < NCH; ++c) {
-          const int cc = (c + sw) % NCH;
-          const int d0 = QF == QF_FP8 ? 16 * cc : 32 * cc;
-          const uint4 ck = *reinterpret_cast<const uint4 *>(src + cc * 16);
-          const uint4 cv = *reinterpret_cast<const uint4 *>(src + RB + cc * 16);
-          const uint32_t sck = QF == QF_FP8 ? sk[0] : (sk[cc >> 1] >> (16 * (cc & 1)));
-          const uint32_t scv = QF == QF_FP8 ? sv[0] : (sv[cc >> 1] >> (16 * (cc & 1)));
-          dequant16<QF>(ck, sck, d0, rk, sw);
-          dequant16<QF>(cv, scv, d0, rv, sw);
-        }
-      } else {
-        // rows past the visible keys: zeros (their probabilities are zero and
-        // zeros keep P x V finite)
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const int off = (c >> 3) * (128 * 128) + (((c & 7) ^ sw) << 4);
-          *reinterpret_cast<uint4 *>(rk + off) = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4 *>(rv + off) = make_uint4(0, 0, 0, 0);
-        }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(2, 128);
-      if (r == 0) {
-        mbar_arrive(k_full + st);
-        mbar_arrive(v_full + st);
-      }
-#pragma unroll
-      for (int i = 0; i < NSW; ++i) {
-        sk[i] = nk[i];
-        sv[i] = nv[i];
-      }
-    }
-    cp_async_wait<0>();
-    if (*abort_flag && r == 0) {
-      // TMA loads issued by this thread must land before the CTA exits
-      for (int j = max(nc, tma_issued - C::NST); j < tma_issued; ++j) {
-        mbar_wait_drain(k_full + j % C::NST, (j / C::NST) & 1);
-        mbar_wait_drain(v_full + j % C::NST, (j / C::NST) & 1);
-      }
-    }
   }
   } else {
     regs_inc<C::REGS_SOFTMAX>();

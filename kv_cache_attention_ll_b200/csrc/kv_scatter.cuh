@@ -182,3 +182,83 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
 }
 
 }  // namespace llk
+
+namespace llk {
+
+// ---------------------------------------------------------------------------
+// Dequantisation of one layer's held frames into a bf16 view.
+//
+// The LongLive-2.0 explainer (wmrh.cn, sec. 15.2-15.3) stores the history KV
+// cache in FP4 and dequantises it in parallel when it is used. Here the
+// visible rows [0, n_rows) of the layer's 2H planes (K then V) are converted
+// once per attention call into the cache's bf16 view [2H][slots][D], which the
+// bf16 attention kernel then reads through TMA; every query tile of a head
+// shares the converted rows instead of converting them again.
+//   FP8:   e4m3 -> f16 (exact) -> fp32, times the row scale, to bf16 (nearest even)
+//   NVFP4: e2m1 -> f16 and E4M3 block scale -> f16 (both exact); the product has
+//          at most 6 significant bits and lies inside the f16 range, so it is
+//          exact, and so is its bf16 conversion.
+// One thread writes 8 bf16 values (16 bytes); reads and writes are coalesced.
+struct DequantParams {
+  const uint8_t *data;     // codes of all layers
+  const uint8_t *scales;   // scales of all layers
+  uint4 *view;             // [2H][slots][D] bf16
+  long long total_vec;     // 2H * n_rows * D/8
+  int H, D, slots, n_rows;
+  int plane0;              // first plane of the layer: layer * 2H
+};
+
+__device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t two_codes) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(static_cast<uint16_t>(two_codes)));
+  return d;
+}
+__device__ __forceinline__ uint32_t f16x2_of_e2m1x2(uint32_t byte) {
+  uint32_t d;
+  asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(d) : "r"(byte));
+  return d;
+}
+__device__ __forceinline__ uint32_t bf16x2_of_f32(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) {
+  const int vpr = q.D >> 3;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < q.total_vec; i += stride) {
+    const int vec = static_cast<int>(i % vpr);
+    const long long pr = i / vpr;                       // (local plane, row)
+    const int row = static_cast<int>(pr % q.n_rows);
+    const int lp = static_cast<int>(pr / q.n_rows);     // 0 .. 2H-1
+    const long long src_row = static_cast<long long>(q.plane0 + lp) * q.slots + row;
+    uint32_t o[4];
+    if constexpr (FMT == FMT_FP8) {
+      const uint2 c = __ldg(reinterpret_cast<const uint2 *>(q.data + src_row * q.D) + vec);
+      const float s = __ldg(reinterpret_cast<const float *>(q.scales) + src_row);
+      const uint32_t w[2] = {c.x, c.y};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t h2 = f16x2_of_e4m3x2(w[k >> 1] >> (16 * (k & 1)));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h2));
+        o[k] = bf16x2_of_f32(f.x * s, f.y * s);
+      }
+    } else {
+      const uint32_t c = __ldg(reinterpret_cast<const uint32_t *>(q.data + src_row * (q.D / 2)) + vec);
+      const uint32_t sb = __ldg(q.scales + src_row * (q.D / 16) + (vec >> 1));
+      const uint32_t s2 = f16x2_of_e4m3x2(sb * 0x101u);   // the block scale in both halves
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t h2 = f16x2_of_e2m1x2((c >> (8 * k)) & 0xFFu);
+        const __half2 prod = __hmul2(*reinterpret_cast<const __half2 *>(&h2), *reinterpret_cast<const __half2 *>(&s2));
+        const float2 f = __half22float2(prod);
+        o[k] = bf16x2_of_f32(f.x, f.y);
+      }
+    }
+    q.view[(static_cast<long long>(lp) * q.slots + row) * vpr + vec] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace llk

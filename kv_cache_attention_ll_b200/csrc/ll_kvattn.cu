@@ -32,6 +32,8 @@ struct ll_kv_cache {
   size_t scale_plane_bytes;   // bytes of one plane's scales
   std::vector<long long> p;   // frames appended per layer
   CUtensorMap tm_cache;       // bf16 cache planes (D, slots, L*2*H)
+  uint8_t *view;              // quantised caches: bf16 view of one layer [2H][slots][D]
+  CUtensorMap tm_view;        // (D, slots, 2H) over the view
 };
 
 namespace {
@@ -99,31 +101,45 @@ int num_sms(int device) {
   return n > 0 ? n : 148;
 }
 
-template <int D, int QF>
+template <int D>
 ll_status launch_attn(const llk::AttnParams &prm, int grid, cudaStream_t stream) {
-  using C = llk::AttnCfg<D, QF>;
+  using C = llk::AttnCfg<D>;
   static std::atomic<unsigned> configured_mask{0};
   int dev = 0;
   cudaGetDevice(&dev);
   const unsigned bit = 1u << (dev & 31);
   if (!(configured_mask.load() & bit)) {
-    if (cudaFuncSetAttribute(llk::attn_sink_window_kernel<D, QF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(llk::attn_sink_window_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_ALLOC) != cudaSuccess)
       return LL_ERR_CUDA;
     configured_mask.fetch_or(bit);
   }
-  llk::attn_sink_window_kernel<D, QF><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(prm);
+  llk::attn_sink_window_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
 
-template <int D>
-ll_status launch_attn_fmt(ll_kv_dtype dt, const llk::AttnParams &prm, int grid, cudaStream_t stream) {
-  switch (dt) {
-    case LL_KV_BF16: return launch_attn<D, llk::QF_BF16>(prm, grid, stream);
-    case LL_KV_FP8_E4M3: return launch_attn<D, llk::QF_FP8>(prm, grid, stream);
-    case LL_KV_NVFP4: return launch_attn<D, llk::QF_NVFP4>(prm, grid, stream);
-  }
-  return LL_ERR_INVALID_ARG;
+// Quantised caches: the layer's visible rows [0, n_rows) of K and V, dequantised
+// into the cache's bf16 view.
+ll_status launch_dequant(ll_kv_cache *c, int layer, int n_rows, cudaStream_t stream) {
+  if (n_rows <= 0) return LL_OK;
+  llk::DequantParams q;
+  q.data = c->data;
+  q.scales = c->scales;
+  q.view = reinterpret_cast<uint4 *>(c->view);
+  q.H = c->H;
+  q.D = c->D;
+  q.slots = static_cast<int>(c->slots);
+  q.n_rows = n_rows;
+  q.plane0 = layer * 2 * c->H;
+  q.total_vec = static_cast<long long>(2 * c->H) * n_rows * (c->D / 8);
+  long long blocks = (q.total_vec + 255) / 256;
+  const long long cap = static_cast<long long>(num_sms(c->device)) * 8;
+  if (blocks > cap) blocks = cap;
+  if (c->dtype == LL_KV_FP8_E4M3)
+    llk::kv_dequant_kernel<llk::FMT_FP8><<<static_cast<int>(blocks), 256, 0, stream>>>(q);
+  else
+    llk::kv_dequant_kernel<llk::FMT_NVFP4><<<static_cast<int>(blocks), 256, 0, stream>>>(q);
+  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
 
 ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, cudaStream_t stream) {
@@ -200,7 +216,12 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   const size_t scale_off = (data_bytes + 255) & ~size_t(255);
   const size_t scale_bytes = scale_plane * planes;
   const size_t err_off = (scale_off + scale_bytes + 255) & ~size_t(255);
-  const size_t total = err_off + 256;
+  // quantised caches also hold a bf16 view of one layer's K and V planes, the
+  // input of the attention kernel after each call's dequantisation
+  const size_t view_off = err_off + 256;
+  const size_t view_bytes =
+      kv_dtype == LL_KV_BF16 ? 0 : static_cast<size_t>(2 * heads) * slots * head_dim * 2;
+  const size_t total = view_off + view_bytes;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
@@ -224,6 +245,7 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   c->data = c->base;
   c->scales = scale_bytes ? c->base + scale_off : nullptr;
   c->err = reinterpret_cast<unsigned *>(c->base + err_off);
+  c->view = view_bytes ? c->base + view_off : nullptr;
   if (cudaMemset(mem, 0, total) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(mem);
     g_alloc_count.fetch_sub(1);
@@ -231,14 +253,18 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
     return LL_ERR_CUDA;
   }
   std::memset(&c->tm_cache, 0, sizeof(c->tm_cache));
-  if (kv_dtype == LL_KV_BF16) {
-    if (!make_map_3d(&c->tm_cache, c->data, head_dim, slots, planes, static_cast<uint64_t>(head_dim) * 2,
-                     static_cast<uint64_t>(slots) * head_dim * 2, 64, 128, 1)) {
-      cudaFree(mem);
-      g_alloc_count.fetch_sub(1);
-      delete c;
-      return LL_ERR_CUDA;
-    }
+  std::memset(&c->tm_view, 0, sizeof(c->tm_view));
+  const bool map_ok =
+      kv_dtype == LL_KV_BF16
+          ? make_map_3d(&c->tm_cache, c->data, head_dim, slots, planes, static_cast<uint64_t>(head_dim) * 2,
+                        static_cast<uint64_t>(slots) * head_dim * 2, 64, 128, 1)
+          : make_map_3d(&c->tm_view, c->view, head_dim, slots, 2 * heads, static_cast<uint64_t>(head_dim) * 2,
+                        static_cast<uint64_t>(slots) * head_dim * 2, 64, 128, 1);
+  if (!map_ok) {
+    cudaFree(mem);
+    g_alloc_count.fetch_sub(1);
+    delete c;
+    return LL_ERR_CUDA;
   }
   *out = c;
   return LL_OK;
@@ -349,22 +375,26 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   if (!make_act_map(&prm.tm_q, q, Tq, c->H, c->D) || !make_act_map(&prm.tm_kcur, k_cur, Tq, c->H, c->D) ||
       !make_act_map(&prm.tm_vcur, v_cur, Tq, c->H, c->D))
     return LL_ERR_CUDA;
-  prm.tm_cache = c->tm_cache;
+  // quantised caches: the layer's held rows are dequantised into the bf16 view
+  // first, and the kernel reads the view (planes: K heads 0..H-1, V heads H..2H-1)
+  const bool quantised = c->dtype != LL_KV_BF16;
+  prm.tm_cache = quantised ? c->tm_view : c->tm_cache;
   prm.out = static_cast<__nv_bfloat16 *>(out);
   prm.err = c->err;
   prm.H = c->H;
   prm.Tq = Tq;
   prm.n_cache = (s + w) * c->T;
-  prm.plane_k = (layer * 2 + 0) * c->H;
-  prm.plane_v = (layer * 2 + 1) * c->H;
+  prm.plane_k = quantised ? 0 : (layer * 2 + 0) * c->H;
+  prm.plane_v = quantised ? c->H : (layer * 2 + 1) * c->H;
   prm.num_q_tiles = (Tq + 127) / 128;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->D)));
-  prm.qdata = c->data;
-  prm.qscales = c->scales;
-  prm.slots = static_cast<int>(c->slots);
   const int grid = prm.num_q_tiles * c->H;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return c->D == 128 ? launch_attn_fmt<128>(c->dtype, prm, grid, st) : launch_attn_fmt<64>(c->dtype, prm, grid, st);
+  if (quantised) {
+    const ll_status ds = launch_dequant(c, layer, prm.n_cache, st);
+    if (ds != LL_OK) return ds;
+  }
+  return c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
 }
 
 }  // extern "C"
