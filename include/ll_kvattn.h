@@ -163,6 +163,39 @@ LL_API size_t ll_kv_export_bytes(const ll_kv_cache *cache);
 LL_API ll_status ll_kv_cache_export(const ll_kv_cache *cache, int layer, void *host_dst, size_t bytes,
                              ll_stream_t stream);
 
+/* ll_attn_sink_window_noalloc - the attention of ll_attn_sink_window over a
+ *   quantised cache layer (FP8 or NVFP4) held in caller memory, performing no
+ *   device allocation at all. The pages have no counterpart: this entry point
+ *   exists for callers that cannot call cudaMalloc, for example code whose
+ *   device memory is owned entirely by a host framework's pool (a serving
+ *   engine that reserves all memory up front and forbids libraries from
+ *   allocating), or code on a latency-critical path where cudaMalloc's implicit
+ *   device synchronisation is not acceptable.
+ *   Inputs (device pointers, caller-owned): q, k_cur, v_cur [F*T][H][D] bf16;
+ *   layer_codes [2][H][(S+W)*T][row bytes] (K planes, then V planes; row bytes
+ *   D for FP8, D/2 for NVFP4) and layer_scales [2][H][(S+W)*T][...] (fp32 per
+ *   row for FP8, D/16 E4M3 bytes per row for NVFP4) - the layout that
+ *   ll_kv_cache_export writes for one layer (data part, then scale part);
+ *   frames_seen = frames appended to this layer so far (p). Output: out
+ *   [F*T][H][D] bf16. Results equal those of ll_attn_sink_window on a cache
+ *   holding the same bytes.
+ *   Scratch: the dequantised bf16 view of the layer, 2*H*(S+W)*T*D*2 bytes,
+ *   lives in a file-scope device array of LL_NOALLOC_SCRATCH_BYTES that every
+ *   GPU loading the library holds until exit. Larger geometries are rejected
+ *   with LL_ERR_INVALID_ARG before anything is enqueued. All calls share that
+ *   array and it keeps the last call's contents, so calls that overlap on the
+ *   GPU (different streams, or different host threads, on one device) race:
+ *   order them. The first call on a device looks up the array's device
+ *   address (once per device, with that device current); make that first call
+ *   before any stream capture. No status word is written by this path.     */
+#define LL_NOALLOC_SCRATCH_BYTES (16u << 20)
+LL_API ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const void *v_cur,
+                                             const void *layer_codes, const void *layer_scales,
+                                             ll_kv_dtype kv_dtype, int heads, int head_dim,
+                                             int tokens_per_frame, int frames_per_chunk, int sink_frames,
+                                             int window_frames, long long frames_seen, void *out,
+                                             ll_stream_t stream);
+
 /* Device-side status word of the cache's kernels: 0 = fine; otherwise a
  * bounded wait inside a kernel gave up (code in the low byte, kernel id in
  * the next byte). Reading synchronises `stream`; `clear` resets it to 0.

@@ -39,6 +39,7 @@ _sig = {
     "ll_kv_export_bytes": (_sz, [_vp]),
     "ll_kv_cache_export": (_i, [_vp, _i, _vp, _sz, _vp]),
     "ll_debug_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint), _i, _vp]),
+    "ll_attn_sink_window_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _ll, _vp, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -171,6 +172,29 @@ def ll_debug_status(cache: KVCache, clear: bool = False, stream=None) -> int:
     if st not in (LL_OK, LL_ERR_TIMEOUT):
         _check(st, "ll_debug_status")
     return w.value
+
+
+def ll_attn_sink_window_noalloc(q, k_cur, v_cur, layer_codes, layer_scales, kv_dtype, heads: int, head_dim: int,
+                                tokens_per_frame: int, frames_per_chunk: int, sink_frames: int, window_frames: int,
+                                frames_seen: int, out, stream=None):
+    """Attention over one quantised cache layer held in caller memory, with no
+    device allocation (the scratch is a static device array of the library).
+    layer_codes / layer_scales: device buffers (uint8 tensors or pointers) in
+    the layout ll_kv_cache_export writes for one layer."""
+    dt = _DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    _check(_lib.ll_attn_sink_window_noalloc(_ptr(q), _ptr(k_cur), _ptr(v_cur), _raw_ptr(layer_codes),
+                                            _raw_ptr(layer_scales), dt, heads, head_dim, tokens_per_frame,
+                                            frames_per_chunk, sink_frames, window_frames, frames_seen, _ptr(out),
+                                            _stream(stream)), "ll_attn_sink_window_noalloc")
+
+
+def _raw_ptr(x) -> int:
+    """Device pointer of a byte buffer (any dtype, contiguous CUDA tensor) or an int."""
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError("buffers must be contiguous CUDA tensors")
+    return x.data_ptr()
 
 
 def raw_lib():

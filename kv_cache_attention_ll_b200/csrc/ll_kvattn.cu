@@ -397,4 +397,122 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   return c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
 }
 
+// ---------------------------------------------------------------------------
+// No-allocation entry point. Its scratch (the dequantised bf16 view of one
+// layer) is this file-scope device array, so the call needs no cudaMalloc. In
+// host code the name is only a stand-in: its device address is looked up once
+// per device with cudaGetSymbolAddress (with that device current) and passed
+// to the kernels.
+static __device__ __align__(256) uint8_t g_noalloc_view[LL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_addr[kMaxDevices] = {};
+
+// device address of g_noalloc_view on the current device (nullptr on failure)
+void *noalloc_scratch(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_view) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    g_noalloc_addr[dev] = ptr;
+  }
+  return g_noalloc_addr[dev];
+}
+}  // namespace
+
+ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const void *v_cur, const void *layer_codes,
+                                      const void *layer_scales, ll_kv_dtype kv_dtype, int heads, int head_dim,
+                                      int tokens_per_frame, int frames_per_chunk, int sink_frames, int window_frames,
+                                      long long frames_seen, void *out, ll_stream_t stream) {
+  if (!q || !k_cur || !v_cur || !layer_codes || !layer_scales || !out) return LL_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out) || !aligned16(layer_codes) ||
+      !aligned16(layer_scales))
+    return LL_ERR_INVALID_ARG;
+  if (out == q || out == k_cur || out == v_cur) return LL_ERR_INVALID_ARG;
+  if (kv_dtype != LL_KV_FP8_E4M3 && kv_dtype != LL_KV_NVFP4) return LL_ERR_INVALID_ARG;
+  if (heads < 1 || tokens_per_frame < 1 || frames_per_chunk < 1 || (head_dim != 64 && head_dim != 128))
+    return LL_ERR_INVALID_ARG;
+  if (sink_frames < 0 || window_frames < 0 || sink_frames + window_frames < 1 || frames_seen < 0)
+    return LL_ERR_INVALID_ARG;
+  const long long slots = static_cast<long long>(sink_frames + window_frames) * tokens_per_frame;
+  const long long tq = static_cast<long long>(frames_per_chunk) * tokens_per_frame;
+  if (slots >= (1ll << 31) || tq >= (1ll << 31)) return LL_ERR_INVALID_ARG;
+  // the view of the layer must fit the static scratch
+  const unsigned long long view_bytes = 2ull * heads * static_cast<unsigned long long>(slots) * head_dim * 2;
+  if (view_bytes > LL_NOALLOC_SCRATCH_BYTES) return LL_ERR_INVALID_ARG;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
+  uint8_t *view = static_cast<uint8_t *>(noalloc_scratch(dev));
+  if (!view) return LL_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  // held context, as for a cache whose layer counter is frames_seen
+  const long long s_held = frames_seen < sink_frames ? frames_seen : sink_frames;
+  long long w_held = frames_seen - sink_frames;
+  if (w_held < 0) w_held = 0;
+  if (w_held > window_frames) w_held = window_frames;
+  const int n_cache = static_cast<int>((s_held + w_held) * tokens_per_frame);
+  const int Tq = static_cast<int>(tq);
+
+  // 1) dequantise the held rows into the view; the rows the ragged last tile
+  //    also reads, [n_cache, min(slots, 128 * ceil(n_cache / 128))), are cleared
+  //    so that they are finite (the array keeps the previous call's contents)
+  if (n_cache > 0) {
+    llk::DequantParams dq;
+    dq.data = static_cast<const uint8_t *>(layer_codes);
+    dq.scales = static_cast<const uint8_t *>(layer_scales);
+    dq.view = reinterpret_cast<uint4 *>(view);
+    dq.H = heads;
+    dq.D = head_dim;
+    dq.slots = static_cast<int>(slots);
+    dq.n_rows = n_cache;
+    dq.plane0 = 0;
+    dq.total_vec = static_cast<long long>(2 * heads) * n_cache * (head_dim / 8);
+    long long blocks = (dq.total_vec + 255) / 256;
+    const long long cap = static_cast<long long>(num_sms(dev)) * 8;
+    if (blocks > cap) blocks = cap;
+    if (kv_dtype == LL_KV_FP8_E4M3)
+      llk::kv_dequant_kernel<llk::FMT_FP8><<<static_cast<int>(blocks), 256, 0, st>>>(dq);
+    else
+      llk::kv_dequant_kernel<llk::FMT_NVFP4><<<static_cast<int>(blocks), 256, 0, st>>>(dq);
+    if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
+    long long tail_end = (static_cast<long long>(n_cache) + 127) / 128 * 128;
+    if (tail_end > slots) tail_end = slots;
+    if (tail_end > n_cache) {
+      const size_t row_b = static_cast<size_t>(head_dim) * 2;
+      if (cudaMemset2DAsync(view + n_cache * row_b, static_cast<size_t>(slots) * row_b, 0,
+                            static_cast<size_t>(tail_end - n_cache) * row_b, static_cast<size_t>(2 * heads),
+                            st) != cudaSuccess)
+        return LL_ERR_CUDA;
+    }
+  }
+
+  // 2) the bf16 attention kernel over the view (planes: K heads 0..H-1, V heads H..2H-1)
+  llk::AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!make_act_map(&prm.tm_q, q, Tq, heads, head_dim) || !make_act_map(&prm.tm_kcur, k_cur, Tq, heads, head_dim) ||
+      !make_act_map(&prm.tm_vcur, v_cur, Tq, heads, head_dim) ||
+      !make_map_3d(&prm.tm_cache, view, head_dim, slots, 2 * heads, static_cast<uint64_t>(head_dim) * 2,
+                   static_cast<uint64_t>(slots) * head_dim * 2, 64, 128, 1))
+    return LL_ERR_CUDA;
+  prm.out = static_cast<__nv_bfloat16 *>(out);
+  prm.err = nullptr;
+  prm.H = heads;
+  prm.Tq = Tq;
+  prm.n_cache = n_cache;
+  prm.plane_k = 0;
+  prm.plane_v = heads;
+  prm.num_q_tiles = (Tq + 127) / 128;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
+  const int grid = prm.num_q_tiles * heads;
+  return head_dim == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
+}
+
 }  // extern "C"
