@@ -47,8 +47,8 @@ ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out
 # ncu DRAM traffic of one attention launch at this shape and the kernel sources it
 # was taken with (profiles/attn_sink_window_wan1.3b.md); reported only while the
 # kernel is unchanged.
-ATTN_TRAFFIC = 168.16e6        # mean of the two captured launches (168.0 MB, 168.3 MB)
-ATTN_TRAFFIC_SRC_SHA = "35c954d108bd0b68"
+ATTN_TRAFFIC = 165.49e6        # mean of the two captured launches (167.6 MB, 163.4 MB)
+ATTN_TRAFFIC_SRC_SHA = "c32deeadcbd0c5a8"
 
 
 def _peaks():

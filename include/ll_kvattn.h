@@ -202,6 +202,18 @@ LL_API ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, c
  * A non-zero word also makes this call return LL_ERR_TIMEOUT.              */
 LL_API ll_status ll_debug_status(ll_kv_cache *cache, unsigned int *word, int clear, ll_stream_t stream);
 
+/* Self-test of the in-kernel failure path: launches one thread that waits, with
+ * the kernels' bounded mbarrier wait, on a barrier that nothing ever completes.
+ * After the wait limit (about a second) the kernel records the timeout in the
+ * cache's status word and returns; read it with ll_debug_status (expect
+ * LL_ERR_TIMEOUT). The context stays usable. Faults nothing, hangs nothing.   */
+LL_API ll_status ll_debug_wait_selftest(ll_kv_cache *cache, ll_stream_t stream);
+
+/* Test hook: when the environment variable LL_KVATTN_TEST_FAIL_ALLOC is set to
+ * a non-empty value other than "0", ll_kv_cache_create fails as if the device
+ * allocation had failed (LL_ERR_OOM), before any CUDA call, releasing
+ * everything it had set up.                                                   */
+
 #ifdef __cplusplus
 }
 #endif

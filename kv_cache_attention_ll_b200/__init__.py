@@ -6,7 +6,7 @@ must be CUDA, bf16, contiguous, 16-byte aligned, token-major [tokens][H][D].
 Raw integer device pointers are accepted too.
 
 Importing this module loads the in-tree library and fails loudly if it is
-missing (build it with `python -m kv_cache_attention_ll_b200.build`); there is
+missing (build it with `python kv_cache_attention_ll_b200/build.py`); there is
 no fallback path.
 """
 from __future__ import annotations
@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libll_kvattn.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build the CUDA library first "
-                      "(python -m kv_cache_attention_ll_b200.build); there is no fallback")
+                      "(python kv_cache_attention_ll_b200/build.py); there is no fallback")
 _lib = ctypes.CDLL(LIB_PATH)
 
 LL_KV_BF16, LL_KV_FP8_E4M3, LL_KV_NVFP4 = 0, 1, 2
@@ -40,6 +40,7 @@ _sig = {
     "ll_kv_cache_export": (_i, [_vp, _i, _vp, _sz, _vp]),
     "ll_debug_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint), _i, _vp]),
     "ll_attn_sink_window_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _ll, _vp, _vp]),
+    "ll_debug_wait_selftest": (_i, [_vp, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -195,6 +196,10 @@ def _raw_ptr(x) -> int:
     if not x.is_cuda or not x.is_contiguous():
         raise ValueError("buffers must be contiguous CUDA tensors")
     return x.data_ptr()
+
+
+def ll_debug_wait_selftest(cache: KVCache, stream=None):
+    _check(_lib.ll_debug_wait_selftest(cache.handle, _stream(stream)), "ll_debug_wait_selftest")
 
 
 def raw_lib():

@@ -1,5 +1,5 @@
 """Build step of the CUDA library: compiles csrc/ into libll_kvattn.so for
-sm_100a, in-tree, next to this file. Run `python -m kv_cache_attention_ll_b200.build`
+sm_100a, in-tree, next to this file. Run `python kv_cache_attention_ll_b200/build.py`
 or call build(); the Python binding loads the result and refuses to run
 without it."""
 from __future__ import annotations

@@ -8,6 +8,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -39,6 +40,11 @@ struct ll_kv_cache {
 namespace {
 
 std::atomic<long long> g_alloc_count{0};
+
+bool test_fail_alloc() {
+  const char *v = std::getenv("LL_KVATTN_TEST_FAIL_ALLOC");
+  return v && v[0] && !(v[0] == '0' && v[1] == 0);
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -223,6 +229,7 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
       kv_dtype == LL_KV_BF16 ? 0 : static_cast<size_t>(2 * heads) * slots * head_dim * 2;
   const size_t total = view_off + view_bytes;
 
+  if (test_fail_alloc()) return LL_ERR_OOM;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
   ll_kv_cache *c = new (std::nothrow) ll_kv_cache();
@@ -395,6 +402,25 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
     if (ds != LL_OK) return ds;
   }
   return c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
+}
+
+// ---------------------------------------------------------------------------
+// Self-test of the bounded wait: one thread waits on a barrier nothing completes.
+namespace llk {
+__global__ void wait_selftest_kernel(unsigned *err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  mbar_init(&bar, 1);
+  abort_flag = 0;
+  fence_mbar_init();
+  mbar_wait(&bar, 0, &abort_flag, err, KID_SELFTEST);
+}
+}  // namespace llk
+
+extern "C" ll_status ll_debug_wait_selftest(ll_kv_cache *c, ll_stream_t stream) {
+  if (!c) return LL_ERR_INVALID_ARG;
+  llk::wait_selftest_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c->err);
+  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------

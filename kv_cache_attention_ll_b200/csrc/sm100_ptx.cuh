@@ -15,6 +15,7 @@ enum : unsigned {
   ERR_WAIT_TIMEOUT = 1u,
   KID_ATTN = 1u << 8,
   KID_SCATTER = 2u << 8,
+  KID_SELFTEST = 3u << 8,
 };
 
 // A wait that is not satisfied after this many SM clocks (~1.1 s at 1.9 GHz)

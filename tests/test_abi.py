@@ -64,3 +64,23 @@ def test_calls_reject_null_cache():
     assert lib.ll_kv_cache_destroy(None) == ll.LL_OK
     assert lib.ll_kv_export_bytes(None) == 0
     assert lib.ll_allocation_count() == 0
+
+
+def test_allocation_failure_hook_reports_oom_and_leaks_nothing():
+    """Host-side fault injection: the test hook makes create fail as if the
+    device allocation had failed; nothing is held afterwards."""
+    import os
+    import kv_cache_attention_ll_b200 as ll
+    lib = ll.raw_lib()
+    before = lib.ll_allocation_count()
+    os.environ["LL_KVATTN_TEST_FAIL_ALLOC"] = "1"
+    try:
+        h = ctypes.c_void_p(1234)
+        assert lib.ll_kv_cache_create(1, 2, 64, 16, 3, 3, 6, 0, ctypes.byref(h)) == ll.LL_ERR_OOM
+        assert h.value is None
+        with pytest.raises(ll.LLError) as e:
+            ll.ll_kv_cache_create(1, 2, 64, 16, 3, 3, 6)
+        assert e.value.status == ll.LL_ERR_OOM
+    finally:
+        del os.environ["LL_KVATTN_TEST_FAIL_ALLOC"]
+    assert lib.ll_allocation_count() == before
