@@ -47,8 +47,8 @@ ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out
 # ncu DRAM traffic of one attention launch at this shape and the kernel sources it
 # was taken with (profiles/attn_sink_window_wan1.3b.md); reported only while the
 # kernel is unchanged.
-ATTN_TRAFFIC = 165.49e6        # mean of the two captured launches (167.6 MB, 163.4 MB)
-ATTN_TRAFFIC_SRC_SHA = "c32deeadcbd0c5a8"
+ATTN_TRAFFIC = 165.80e6        # mean of the two captured launches (167.85 MB, 163.75 MB)
+ATTN_TRAFFIC_SRC_SHA = "9b360afb25ef9eca"
 
 
 def _peaks():
@@ -260,14 +260,14 @@ def run_ours(args, world, rank, local):
     attn_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(L)]
                for _ in range(args.steps)]
 
-    def step(ev=None):
+    def step(ev=None, st=stream):
         for l in range(L):
             if ev is not None:
-                ev[l][0].record(stream)
-            ll.ll_attn_sink_window(qs[l], ks[l], vs[l], cache, l, outs[l], stream)
+                ev[l][0].record(st)
+            ll.ll_attn_sink_window(qs[l], ks[l], vs[l], cache, l, outs[l], st)
             if ev is not None:
-                ev[l][1].record(stream)
-            ll.ll_kv_append(cache, l, ks[l], vs[l], stream)
+                ev[l][1].record(st)
+            ll.ll_kv_append(cache, l, ks[l], vs[l], st)
 
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     # clocks are sampled from the start of the warm-up to the end of the timed steps
@@ -282,7 +282,28 @@ def run_ours(args, world, rank, local):
             step(attn_ev[i])
         e1.record(stream)
         torch.cuda.synchronize(dev)
-    total_ms = e0.elapsed_time(e1)
+        total_ms = e0.elapsed_time(e1)
+        # ---- the same chunk step captured once in a CUDA graph and replayed:
+        # the kernels read the frame counters from device memory, so every
+        # replay is the next chunk (counters advance, the ring moves)
+        graph_leg = None
+        if not args.no_graph:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                step(st=torch.cuda.current_stream(dev))
+            for _ in range(3):
+                gr.replay()
+            torch.cuda.synchronize(dev)
+            _barrier(world)
+            e0.record(stream)
+            for _ in range(args.steps):
+                gr.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            g_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+            graph_leg = {"ms_per_step": g_ms, "value": world * ATTN_FLOP * L / (g_ms * 1e-3) / 1e12,
+                         "launches_per_step": 2 * L}
+            del gr
     attn_ms = [a.elapsed_time(b) for ev in attn_ev for a, b in ev]
     _barrier(world)
     total_ms = _max_over_ranks(total_ms, world)
@@ -492,6 +513,7 @@ def run_ours(args, world, rank, local):
                     "gbs": recache_bytes(L) / (rec_ms * 1e-3) / 1e9,
                     "frac_hbm": recache_bytes(L) / (rec_ms * 1e-3) / 1e9 / peak_gbs},
         "e2e": e2e,
+        "cuda_graph_step": graph_leg,
         "gpu_launches": 2 * L * args.steps,
         "clocks": clk.summary(),
         "cpu_baseline": cpu,
@@ -514,6 +536,7 @@ def main():
     ap.add_argument("--no-quant", action="store_true", help="skip the FP8 / NVFP4 cache leg")
     ap.add_argument("--quant-steps", type=int, default=10)
     ap.add_argument("--no-sweep", action="store_true", help="skip the window sweep / full-causal leg")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
     ap.add_argument("--layers", type=int, default=30, help="stack depth (30 = the Wan-1.3B stack)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="CPU seconds the reference arm spends in total (bounded sample per step)")

@@ -82,10 +82,13 @@ typedef enum {
  *   FP8 [H][(S+W)*T] fp32; NVFP4 [H][(S+W)*T][D/16] E4M3 bytes; and a bf16
  *   view of ONE layer's K and V planes (2*H*(S+W)*T*D*2 bytes) that each
  *   ll_attn_sink_window call refills with the dequantised held frames.
- *   The memory is zero-filled at create; frame counters start at 0.
+ *   The memory is zero-filled at create; frame counters start at 0. The
+ *   frame counter p of each layer lives in device memory: the kernels read it
+ *   and ll_kv_append advances it, so calls recorded in a CUDA graph (stream
+ *   capture) stay right when the graph is replayed chunk after chunk.
  *   Supported: layers, heads, tokens_per_frame, frames_per_chunk >= 1;
  *   head_dim in {64, 128}; sink_frames >= 0, window_frames >= 0,
- *   sink_frames + window_frames >= 1; (S+W)*T and F*T < 2^31.
+ *   sink_frames + window_frames >= 1; (S+W)*T and F*T < 2^31; T*H*D/8 < 2^30.
  *   Returns LL_ERR_INVALID_ARG on a bad parameter or null `out`,
  *   LL_ERR_OOM if the allocation fails, LL_ERR_CUDA if no device is usable.
  *   On success *out owns the memory until ll_kv_cache_destroy.           */
@@ -98,7 +101,10 @@ LL_API ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tok
  *   Frame f = p..p+F-1 (p = frames appended to this layer so far) goes to slot
  *   f if f < S; otherwise, if f >= p+F-W, to ring slot S + ((f-S) mod W),
  *   overwriting (evicting) the oldest window frame; other frames (only when
- *   W < F) are not stored. Quantised caches quantise here. Then p += F.
+ *   W < F) are not stored. Quantised caches quantise here. Then p += F, on
+ *   the device, at the end of the launch (p is read from device memory).
+ *   An append enqueued inside a stream capture ends the host's knowledge of
+ *   p (see ll_kv_cache_info and ll_kv_recache_write).
  *   Pages: dpshk.com sec. 五/六; techwalker.com sec. 六.                    */
 LL_API ll_status ll_kv_append(ll_kv_cache *cache, int layer, const void *k_cur, const void *v_cur,
                        ll_stream_t stream);
@@ -109,8 +115,12 @@ LL_API ll_status ll_kv_append(ll_kv_cache *cache, int layer, const void *k_cur, 
  *   single layer or L for all layers; frame i of the source replaces logical
  *   frame first_frame+i of the held context, whose logical order is: sink
  *   frames 0..s-1, then window frames oldest to newest (s = min(p,S),
- *   w = min(W, max(0, p-S))). Requires 0 <= first_frame, num_frames >= 1 and
- *   first_frame + num_frames <= s + w of every addressed layer.
+ *   w = min(W, max(0, p-S)), p the layer's own counter). Requires
+ *   0 <= first_frame, num_frames >= 1, first_frame + num_frames <= S + W
+ *   (else LL_ERR_INVALID_ARG) and <= s + w of every addressed layer: checked
+ *   by the host (LL_ERR_INVALID_ARG) while it knows p; after a captured
+ *   append, by the kernel, which then writes nothing to such a layer and sets
+ *   ERR_RANGE in the status word (ll_debug_status).
  *   Frame counters and the ring position are unchanged.
  *   Sink + window is the default context (dpshk.com sec. 三.3); first_frame = S,
  *   num_frames = W gives the window-only variant with the sink unchanged
@@ -147,7 +157,9 @@ LL_API ll_status ll_kv_cache_destroy(ll_kv_cache *cache);
 LL_API const char *ll_status_string(ll_status status);
 
 /* Frames appended so far to `layer` (p) and the cache's total device bytes
- * (all layers, data + scales). Either output pointer may be NULL.           */
+ * (all layers, data + scales). Either output pointer may be NULL. Once an
+ * append has been enqueued inside a stream capture, p is read from the device
+ * after a device-wide synchronisation (do not call it while capturing).     */
 LL_API ll_status ll_kv_cache_info(const ll_kv_cache *cache, int layer, long long *frames_seen,
                            size_t *device_bytes);
 
@@ -196,10 +208,13 @@ LL_API ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, c
                                              int window_frames, long long frames_seen, void *out,
                                              ll_stream_t stream);
 
-/* Device-side status word of the cache's kernels: 0 = fine; otherwise a
- * bounded wait inside a kernel gave up (code in the low byte, kernel id in
- * the next byte). Reading synchronises `stream`; `clear` resets it to 0.
- * A non-zero word also makes this call return LL_ERR_TIMEOUT.              */
+/* Device-side status word of the cache's kernels: 0 = fine; otherwise OR-ed
+ * flags, reasons in the low byte (1 = a bounded in-kernel wait gave up,
+ * 2 = a recache addressed frames a layer does not hold) and the reporting
+ * kernels in the next (1 = attention, 2 = append/recache, 4 = self-test).
+ * Reading synchronises `stream`; `clear` resets it to 0. The call returns
+ * LL_ERR_TIMEOUT if reason 1 is set, LL_ERR_INVALID_ARG for any other
+ * non-zero word, LL_OK for 0; *word is filled in all three cases.          */
 LL_API ll_status ll_debug_status(ll_kv_cache *cache, unsigned int *word, int clear, ll_stream_t stream);
 
 /* Self-test of the in-kernel failure path: launches one thread that waits, with

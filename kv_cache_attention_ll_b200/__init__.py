@@ -168,9 +168,12 @@ def ll_kv_cache_export(cache: KVCache, layer: int, stream=None) -> bytes:
 
 
 def ll_debug_status(cache: KVCache, clear: bool = False, stream=None) -> int:
+    """The cache's device status word (0 = fine); see ll_debug_status in the header."""
+    if not cache.handle:
+        raise ValueError("closed cache")
     w = ctypes.c_uint()
     st = _lib.ll_debug_status(cache.handle, ctypes.byref(w), int(clear), _stream(stream))
-    if st not in (LL_OK, LL_ERR_TIMEOUT):
+    if st not in (LL_OK, LL_ERR_TIMEOUT, LL_ERR_INVALID_ARG):   # the last two report a non-zero word
         _check(st, "ll_debug_status")
     return w.value
 

@@ -46,9 +46,11 @@ struct AttnParams {
   CUtensorMap tm_cache;  // (D, slots, L*2*H) bf16, box (64, 128, 1)
   __nv_bfloat16 *out;    // [Tq][H][D]
   unsigned *err;         // status word (see sm100_ptx.cuh)
+  const long long *frames;  // this layer's device frame counter p, or null: then n_cache is used
   int H;
   int Tq;
-  int n_cache;           // visible cache keys: slots [0, n_cache)
+  int n_cache;           // visible cache keys when frames is null: slots [0, n_cache)
+  int S, W, T;           // sink frames, window frames, tokens per frame (with frames)
   int plane_k;           // (l*2 + 0) * H : plane of head 0 of this layer's K
   int plane_v;           // (l*2 + 1) * H
   int num_q_tiles;
@@ -95,6 +97,18 @@ struct AttnCfg {
 // FMA-pipe polynomials balances the two pipes.
 constexpr unsigned kPolyPairs = 0x88u;
 
+// Visible cache keys: (s + w) * T with s = min(p, S), w = min(W, max(0, p - S)),
+// p read from the layer's device counter (advanced by the append kernel), so
+// the same launch is right for any p, as when a captured graph is replayed.
+__device__ __forceinline__ int visible_cache_keys(const AttnParams &prm) {
+  if (!prm.frames) return prm.n_cache;
+  const long long p = __ldcg(prm.frames);
+  const long long s = p < prm.S ? p : prm.S;
+  long long w = p - prm.S;
+  w = w < 0 ? 0 : (w > prm.W ? prm.W : w);
+  return static_cast<int>((s + w) * prm.T);
+}
+
 __device__ __forceinline__ int tile_valid(int j, int nc, int n_cache, int Tq) {
   if (j < nc) return min(128, n_cache - j * 128);
   return min(128, Tq - (j - nc) * 128);
@@ -128,7 +142,8 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
   const int unit = blockIdx.x;
   const int h = unit / prm.num_q_tiles;
   const int q0 = (unit % prm.num_q_tiles) * C::BM;
-  const int nc = (prm.n_cache + C::BN - 1) / C::BN;
+  const int n_cache = visible_cache_keys(prm);
+  const int nc = (n_cache + C::BN - 1) / C::BN;
   const int nown = (prm.Tq + C::BN - 1) / C::BN;
   const int n_tiles = nc + nown;
 
@@ -312,7 +327,7 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
       uint32_t sr[128];
       tmem_ld64(TM_S(g) + lane_off, sr);
       tmem_ld64(TM_S(g) + lane_off + 64, sr + 64);
-      const int valid = tile_valid(j, nc, prm.n_cache, prm.Tq);
+      const int valid = tile_valid(j, nc, n_cache, prm.Tq);
       if (valid < 128) {
 #pragma unroll
         for (int e = 0; e < 128; ++e)

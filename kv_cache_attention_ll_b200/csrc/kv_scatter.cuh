@@ -9,15 +9,21 @@
 //   recache (dpshk.com sec. 三.5; techwalker.com LONGLIVE article sec. 六): logical
 //            frame k of the held context -> k if k < s, else the ring slot of
 //            absolute frame p - w + (k - s).
-// One thread moves one 16-byte vector (8 values) of K and the same vector of V;
-// the D/8 threads of one (token, head) row are consecutive lanes, so reads are
-// fully coalesced and each row is written as one contiguous 128/256-byte run.
+// Grid: blockIdx.x = one (source layer, source frame) pair, blockIdx.y strides
+// over that frame's T*H*D/8 16-byte vectors. Everything that depends on the
+// layer's frame counter (the destination slot, or that nothing is stored) is
+// decided once per block. One thread moves one vector (8 values) of K and the
+// same vector of V; the D/8 threads of one (token, head) row are consecutive
+// lanes, so reads are fully coalesced and each row is written as one
+// contiguous 128/256-byte run.
 // Quantising formats reduce the row (FP8) or the 16-value block (NVFP4) with
 // lane shuffles inside that group and write codes + scales.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
+
+#include "sm100_ptx.cuh"
 
 namespace llk {
 
@@ -29,26 +35,38 @@ struct ScatterParams {
   const uint4 *src_v;
   uint8_t *data;             // cache data base (all layers)
   uint8_t *scales;           // cache scale base (quantised formats) or null
-  long long total_vec;       // n_layers * n_frames*T * H * (D/8)
+  int frame_vec;             // T * H * (D/8): vectors of one frame (< 2^30)
   int H, D, T, slots;        // slots = (S+W)*T per plane
   int layer0;                // first destination layer
   int n_frames;              // frames per source layer
   int mode;                  // ScatterMode
   int S, W, F;               // cache geometry
-  int p;                     // frames appended before (append) / held state (recache)
-  int s, w, first;           // recache: held sink/window frames, first logical frame
+  int first;                 // recache: first logical frame
+  long long *frames;         // per-layer frame counters p (device); append advances its layer's by F
+  unsigned *done;            // per-layer count of finished append blocks (zero between launches)
+  unsigned *err;             // status word: recache beyond the held frames is flagged there
 };
 
-__device__ __forceinline__ int scatter_slot(const ScatterParams &q, int fi) {
+// Only whether p < S and the ring position (p - S) mod W matter once p >= S + W,
+// so very long rollouts fold into int range without changing any slot.
+__device__ __forceinline__ int fold_frames(long long p, int S, int W) {
+  if (p <= (1ll << 30)) return static_cast<int>(p);
+  if (W == 0) return S + W;
+  return S + W + static_cast<int>((p - S) % W);
+}
+
+// Destination frame slot of source frame fi, or -1 when it is not stored.
+// p: folded counter of the layer; s, w: its held sink and window frames.
+__device__ __forceinline__ int scatter_slot(const ScatterParams &q, int p, int s, int w, int fi) {
   if (q.mode == SCATTER_APPEND) {
-    const int f = q.p + fi;
+    const int f = p + fi;
     if (f < q.S) return f;
-    if (q.W > 0 && f >= q.p + q.F - q.W) return q.S + (f - q.S) % q.W;
+    if (q.W > 0 && f >= p + q.F - q.W) return q.S + (f - q.S) % q.W;
     return -1;
   }
   const int k = q.first + fi;
-  if (k < q.s) return k;
-  const int a = q.p - q.w + (k - q.s);
+  if (k < s) return k;
+  const int a = p - w + (k - s);
   return q.S + (a - q.S) % q.W;
 }
 
@@ -98,30 +116,38 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&x)[8]) {
 template <int FMT>
 __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) {
   const int vpr = q.D >> 3;                    // vectors per (token, head) row: 8 or 16
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  // warp-uniform trip count: every lane runs every iteration so that the
-  // row-group shuffles of the quantising formats always see all 32 lanes
-  for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x; base < q.total_vec; base += stride) {
-    const long long i = base + threadIdx.x;
-    const bool in = i < q.total_vec;
-    const long long ic = in ? i : 0;
-    const int vec = static_cast<int>(ic % vpr);
-    const long long row = ic / vpr;                         // (layer_i, token, head)
-    const int hh = static_cast<int>(row % q.H);
-    const long long lt = row / q.H;                         // (layer_i, token)
-    const int li = static_cast<int>(lt / (static_cast<long long>(q.n_frames) * q.T));
-    const int tok = static_cast<int>(lt % (static_cast<long long>(q.n_frames) * q.T));
-    const int fi = tok / q.T, t = tok % q.T;
-    const int slot = scatter_slot(q, fi);
-    const bool act = in && slot >= 0;
-    const int layer = q.layer0 + li;
+  const int lg_vpr = vpr == 16 ? 4 : 3;
+  const int li = blockIdx.x / q.n_frames;      // source layer
+  const int fi = blockIdx.x % q.n_frames;      // source frame
+  const int layer = q.layer0 + li;
+  // the layer's counter; every block reads it before its own completion count
+  // below, so the append's advance (by the last block) comes after all reads
+  const long long p_raw = __ldcg(q.frames + layer);
+  const int s_held = static_cast<int>(p_raw < q.S ? p_raw : q.S);
+  const int w_held = static_cast<int>(p_raw - q.S < 0 ? 0 : (p_raw - q.S > q.W ? q.W : p_raw - q.S));
+  // recache of frames the layer does not hold: nothing of that layer is written
+  const bool reject = q.mode == SCATTER_RECACHE && q.first + q.n_frames > s_held + w_held;
+  if (reject && fi == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(q.err, KID_SCATTER | ERR_RANGE);
+  const int slot = reject ? -1 : scatter_slot(q, fold_frames(p_raw, q.S, q.W), s_held, w_held, fi);
+  const long long src0 = static_cast<long long>(blockIdx.x) * q.frame_vec;   // first vector of the frame
+  const int stride = gridDim.y * blockDim.x;
+  // block-uniform trip count (slot is uniform too): every lane runs every
+  // iteration, so the row-group shuffles of the quantising formats see all 32
+  for (int base = slot < 0 ? q.frame_vec : blockIdx.y * blockDim.x; base < q.frame_vec; base += stride) {
+    const int i = base + threadIdx.x;
+    const bool act = i < q.frame_vec;
+    const int ic = act ? i : 0;
+    const int vec = ic & (vpr - 1);
+    const int row = ic >> lg_vpr;                           // token * H + head
+    const int t = row / q.H;
+    const int hh = row - t * q.H;
     const long long plane_k = (static_cast<long long>(layer) * 2 + 0) * q.H + hh;
     const long long plane_v = plane_k + q.H;
     const long long drow = static_cast<long long>(slot) * q.T + t;   // row inside a plane
     uint4 vk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
     if (act) {
-      vk = __ldg(q.src_k + ic);
-      vv = __ldg(q.src_v + ic);
+      vk = __ldg(q.src_k + src0 + ic);
+      vv = __ldg(q.src_v + src0 + ic);
     }
     if constexpr (FMT == FMT_BF16) {
       if (act) {
@@ -179,6 +205,20 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
       }
     }
   }
+  if (q.mode == SCATTER_APPEND) {
+    // the last block to finish advances the counter; every thread of every
+    // block read it above, before this barrier and its block's increment
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const unsigned prev = atomicAdd(q.done + q.layer0, 1u);
+      if (prev == gridDim.x * gridDim.y - 1) {
+        q.frames[q.layer0] = p_raw + q.F;
+        q.done[q.layer0] = 0;
+        __threadfence();
+      }
+    }
+  }
 }
 
 }  // namespace llk
@@ -203,8 +243,9 @@ struct DequantParams {
   const uint8_t *data;     // codes of all layers
   const uint8_t *scales;   // scales of all layers
   uint4 *view;             // [2H][slots][D] bf16
-  long long total_vec;     // 2H * n_rows * D/8
+  const long long *frames; // the layer's device frame counter, or null: then n_rows is used
   int H, D, slots, n_rows;
+  int S, W, T;             // with frames: rows = (min(p,S) + min(W, max(0, p-S))) * T
   int plane0;              // first plane of the layer: layer * 2H
 };
 
@@ -228,11 +269,20 @@ template <int FMT>
 __global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) {
   const int vpr = q.D >> 3;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < q.total_vec; i += stride) {
+  int n_rows = q.n_rows;
+  if (q.frames) {
+    const long long p = __ldcg(q.frames);
+    const long long s = p < q.S ? p : q.S;
+    long long w = p - q.S;
+    w = w < 0 ? 0 : (w > q.W ? q.W : w);
+    n_rows = static_cast<int>((s + w) * q.T);
+  }
+  const long long total_vec = static_cast<long long>(2 * q.H) * n_rows * vpr;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_vec; i += stride) {
     const int vec = static_cast<int>(i % vpr);
     const long long pr = i / vpr;                       // (local plane, row)
-    const int row = static_cast<int>(pr % q.n_rows);
-    const int lp = static_cast<int>(pr / q.n_rows);     // 0 .. 2H-1
+    const int row = static_cast<int>(pr % n_rows);
+    const int lp = static_cast<int>(pr / n_rows);       // 0 .. 2H-1
     const long long src_row = static_cast<long long>(q.plane0 + lp) * q.slots + row;
     uint32_t o[4];
     if constexpr (FMT == FMT_FP8) {

@@ -1,7 +1,13 @@
 // ll_kvattn.cu - host side of the C ABI declared in include/ll_kvattn.h:
 // the cache object (one device allocation per cache, zero-filled, never grown),
-// argument validation, ring-buffer bookkeeping (host-side frame counters),
-// TMA descriptor setup and the kernel launches.
+// argument validation, TMA descriptor setup and the kernel launches.
+//
+// Frame counters live in device memory: the kernels read a layer's p there and
+// the append kernel advances it, so a captured sequence of calls stays right
+// when it is replayed. The host keeps a mirror for argument checks and
+// ll_kv_cache_info until an append is enqueued inside a stream capture; from
+// then on replays move the device counters without the host seeing them, so
+// info reads the device and recache range checks happen in the kernel.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -31,7 +37,10 @@ struct ll_kv_cache {
   unsigned *err;              // device status word
   size_t data_plane_bytes;    // bytes of one plane's data
   size_t scale_plane_bytes;   // bytes of one plane's scales
-  std::vector<long long> p;   // frames appended per layer
+  std::vector<long long> p;   // host mirror of the frame counters (exact while host_counters)
+  bool host_counters;         // false once an append was enqueued inside a stream capture
+  long long *frames;          // device frame counters [L]
+  unsigned *done;             // device append-completion counts [L]
   CUtensorMap tm_cache;       // bf16 cache planes (D, slots, L*2*H)
   uint8_t *view;              // quantised caches: bf16 view of one layer [2H][slots][D]
   CUtensorMap tm_view;        // (D, slots, 2H) over the view
@@ -77,9 +86,13 @@ bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uin
   return r == CUDA_SUCCESS;
 }
 
-// token-major activation [Tq][H][D] viewed as (D, H, Tq), box (64, 1, 128)
+// key rows per attention tile: every TMA box of keys (and of queries) is 64
+// head-dim columns x kKeyTile rows
+constexpr uint32_t kKeyTile = llk::AttnCfg<128>::BN;
+
+// token-major activation [Tq][H][D] viewed as (D, H, Tq), box (64, 1, kKeyTile)
 bool make_act_map(CUtensorMap *m, const void *p, int Tq, int H, int D) {
-  return make_map_3d(m, p, D, H, Tq, static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(H) * D * 2, 64, 1, 128);
+  return make_map_3d(m, p, D, H, Tq, static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(H) * D * 2, 64, 1, kKeyTile);
 }
 
 void held(const ll_kv_cache *c, int layer, int *s, int *w) {
@@ -89,16 +102,6 @@ void held(const ll_kv_cache *c, int layer, int *s, int *w) {
   if (ww < 0) ww = 0;
   if (ww > c->W) ww = c->W;
   *w = static_cast<int>(ww);
-}
-
-// The frame counter as the kernels see it: only whether p < S and the ring
-// position (p - S) mod W matter once p >= S + W, so very long rollouts are
-// folded into int range without changing any slot.
-int kernel_p(const ll_kv_cache *c, int layer) {
-  const long long p = c->p[layer];
-  if (p <= (1ll << 30)) return static_cast<int>(p);
-  if (c->W == 0) return c->S + c->W;
-  return c->S + c->W + static_cast<int>((p - c->S) % c->W);
 }
 
 int num_sms(int device) {
@@ -124,10 +127,9 @@ ll_status launch_attn(const llk::AttnParams &prm, int grid, cudaStream_t stream)
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
 
-// Quantised caches: the layer's visible rows [0, n_rows) of K and V, dequantised
-// into the cache's bf16 view.
-ll_status launch_dequant(ll_kv_cache *c, int layer, int n_rows, cudaStream_t stream) {
-  if (n_rows <= 0) return LL_OK;
+// Quantised caches: the layer's held rows of K and V (their number follows the
+// layer's device counter), dequantised into the cache's bf16 view.
+ll_status launch_dequant(ll_kv_cache *c, int layer, cudaStream_t stream) {
   llk::DequantParams q;
   q.data = c->data;
   q.scales = c->scales;
@@ -135,10 +137,13 @@ ll_status launch_dequant(ll_kv_cache *c, int layer, int n_rows, cudaStream_t str
   q.H = c->H;
   q.D = c->D;
   q.slots = static_cast<int>(c->slots);
-  q.n_rows = n_rows;
+  q.frames = c->frames + layer;
+  q.n_rows = 0;
+  q.S = c->S;
+  q.W = c->W;
+  q.T = c->T;
   q.plane0 = layer * 2 * c->H;
-  q.total_vec = static_cast<long long>(2 * c->H) * n_rows * (c->D / 8);
-  long long blocks = (q.total_vec + 255) / 256;
+  long long blocks = (static_cast<long long>(2 * c->H) * c->slots * (c->D / 8) + 255) / 256;
   const long long cap = static_cast<long long>(num_sms(c->device)) * 8;
   if (blocks > cap) blocks = cap;
   if (c->dtype == LL_KV_FP8_E4M3)
@@ -148,15 +153,22 @@ ll_status launch_dequant(ll_kv_cache *c, int layer, int n_rows, cudaStream_t str
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
 
-ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, cudaStream_t stream) {
-  if (q.total_vec == 0) return LL_OK;
-  long long blocks = (q.total_vec + 255) / 256;
-  const long long cap = static_cast<long long>(num_sms(c->device)) * 8;
-  if (blocks > cap) blocks = cap;
+// Grid: one x-block per (source layer, source frame) pair, y-blocks striding
+// over the frame's vectors; about 8 blocks of 256 threads per SM in total.
+ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, int n_layers, cudaStream_t stream) {
+  const long long pairs = static_cast<long long>(n_layers) * q.n_frames;
+  if (pairs < 1 || pairs >= (1ll << 31)) return LL_ERR_INVALID_ARG;
+  const long long per_frame_blocks = (q.frame_vec + 255) / 256;
+  const long long target = static_cast<long long>(num_sms(c->device)) * 8;
+  long long gy = (target + pairs - 1) / pairs;
+  if (gy > per_frame_blocks) gy = per_frame_blocks;
+  if (gy > 65535) gy = 65535;
+  if (gy < 1) gy = 1;
+  const dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(gy));
   switch (c->dtype) {
-    case LL_KV_BF16: llk::kv_scatter_kernel<llk::FMT_BF16><<<static_cast<int>(blocks), 256, 0, stream>>>(q); break;
-    case LL_KV_FP8_E4M3: llk::kv_scatter_kernel<llk::FMT_FP8><<<static_cast<int>(blocks), 256, 0, stream>>>(q); break;
-    case LL_KV_NVFP4: llk::kv_scatter_kernel<llk::FMT_NVFP4><<<static_cast<int>(blocks), 256, 0, stream>>>(q); break;
+    case LL_KV_BF16: llk::kv_scatter_kernel<llk::FMT_BF16><<<grid, 256, 0, stream>>>(q); break;
+    case LL_KV_FP8_E4M3: llk::kv_scatter_kernel<llk::FMT_FP8><<<grid, 256, 0, stream>>>(q); break;
+    case LL_KV_NVFP4: llk::kv_scatter_kernel<llk::FMT_NVFP4><<<grid, 256, 0, stream>>>(q); break;
   }
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
@@ -171,10 +183,14 @@ llk::ScatterParams scatter_base(const ll_kv_cache *c, const void *k, const void 
   q.H = c->H;
   q.D = c->D;
   q.T = c->T;
+  q.frame_vec = c->T * c->H * (c->D / 8);
   q.slots = static_cast<int>(c->slots);
   q.S = c->S;
   q.W = c->W;
   q.F = c->F;
+  q.frames = c->frames;
+  q.done = c->done;
+  q.err = c->err;
   return q;
 }
 
@@ -207,6 +223,7 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   const long long slots = static_cast<long long>(sink_frames + window_frames) * tokens_per_frame;
   const long long tq = static_cast<long long>(frames_per_chunk) * tokens_per_frame;
   if (slots >= (1ll << 31) || tq >= (1ll << 31)) return LL_ERR_INVALID_ARG;
+  if (static_cast<long long>(tokens_per_frame) * heads * (head_dim / 8) >= (1ll << 30)) return LL_ERR_INVALID_ARG;
   const long long planes = static_cast<long long>(layers) * 2 * heads;
   if (planes >= (1ll << 31)) return LL_ERR_INVALID_ARG;
 
@@ -224,7 +241,9 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   const size_t err_off = (scale_off + scale_bytes + 255) & ~size_t(255);
   // quantised caches also hold a bf16 view of one layer's K and V planes, the
   // input of the attention kernel after each call's dequantisation
-  const size_t view_off = err_off + 256;
+  const size_t ctr_off = err_off + 256;
+  const size_t ctr_bytes = ((static_cast<size_t>(layers) * 12 + 255) / 256) * 256;   // counters, done counts
+  const size_t view_off = ctr_off + ctr_bytes;
   const size_t view_bytes =
       kv_dtype == LL_KV_BF16 ? 0 : static_cast<size_t>(2 * heads) * slots * head_dim * 2;
   const size_t total = view_off + view_bytes;
@@ -237,6 +256,7 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   c->L = layers; c->H = heads; c->D = head_dim; c->T = tokens_per_frame; c->F = frames_per_chunk;
   c->S = sink_frames; c->W = window_frames; c->dtype = kv_dtype; c->device = dev; c->slots = slots;
   c->p.assign(layers, 0);
+  c->host_counters = true;
   c->data_plane_bytes = data_plane;
   c->scale_plane_bytes = scale_plane;
   void *mem = nullptr;
@@ -252,6 +272,8 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   c->data = c->base;
   c->scales = scale_bytes ? c->base + scale_off : nullptr;
   c->err = reinterpret_cast<unsigned *>(c->base + err_off);
+  c->frames = reinterpret_cast<long long *>(c->base + ctr_off);
+  c->done = reinterpret_cast<unsigned *>(c->base + ctr_off + static_cast<size_t>(layers) * 8);
   c->view = view_bytes ? c->base + view_off : nullptr;
   if (cudaMemset(mem, 0, total) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(mem);
@@ -264,9 +286,9 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   const bool map_ok =
       kv_dtype == LL_KV_BF16
           ? make_map_3d(&c->tm_cache, c->data, head_dim, slots, planes, static_cast<uint64_t>(head_dim) * 2,
-                        static_cast<uint64_t>(slots) * head_dim * 2, 64, 128, 1)
+                        static_cast<uint64_t>(slots) * head_dim * 2, 64, kKeyTile, 1)
           : make_map_3d(&c->tm_view, c->view, head_dim, slots, 2 * heads, static_cast<uint64_t>(head_dim) * 2,
-                        static_cast<uint64_t>(slots) * head_dim * 2, 64, 128, 1);
+                        static_cast<uint64_t>(slots) * head_dim * 2, 64, kKeyTile, 1);
   if (!map_ok) {
     cudaFree(mem);
     g_alloc_count.fetch_sub(1);
@@ -292,7 +314,23 @@ ll_status ll_kv_cache_destroy(ll_kv_cache *c) {
 
 ll_status ll_kv_cache_info(const ll_kv_cache *c, int layer, long long *frames_seen, size_t *device_bytes) {
   if (!c || layer < 0 || layer >= c->L) return LL_ERR_INVALID_ARG;
-  if (frames_seen) *frames_seen = c->p[layer];
+  if (frames_seen) {
+    if (c->host_counters) {
+      *frames_seen = c->p[layer];
+    } else {
+      // replays of captured appends have moved the device counter: wait for all
+      // work on the device, then read it
+      int prev = 0;
+      cudaGetDevice(&prev);
+      if (cudaSetDevice(c->device) != cudaSuccess) return LL_ERR_CUDA;
+      long long v = 0;
+      const bool ok = cudaDeviceSynchronize() == cudaSuccess &&
+                      cudaMemcpy(&v, c->frames + layer, sizeof(v), cudaMemcpyDeviceToHost) == cudaSuccess;
+      cudaSetDevice(prev);
+      if (!ok) return LL_ERR_CUDA;
+      *frames_seen = v;
+    }
+  }
   if (device_bytes) *device_bytes = c->bytes;
   return LL_OK;
 }
@@ -325,21 +363,29 @@ ll_status ll_debug_status(ll_kv_cache *c, unsigned int *word, int clear, ll_stre
   if (cudaStreamSynchronize(s) != cudaSuccess) return LL_ERR_CUDA;
   if (clear && cudaMemsetAsync(c->err, 0, sizeof(unsigned), s) != cudaSuccess) return LL_ERR_CUDA;
   *word = w;
-  return w ? LL_ERR_TIMEOUT : LL_OK;
+  if (w & llk::ERR_WAIT_TIMEOUT) return LL_ERR_TIMEOUT;
+  return w ? LL_ERR_INVALID_ARG : LL_OK;
 }
 
 ll_status ll_kv_append(ll_kv_cache *c, int layer, const void *k_cur, const void *v_cur, ll_stream_t stream) {
   if (!c || layer < 0 || layer >= c->L || !k_cur || !v_cur || !aligned16(k_cur) || !aligned16(v_cur))
     return LL_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return LL_ERR_CUDA;
+  }
   llk::ScatterParams q = scatter_base(c, k_cur, v_cur);
   q.mode = llk::SCATTER_APPEND;
   q.layer0 = layer;
   q.n_frames = c->F;
-  q.p = kernel_p(c, layer);
-  q.total_vec = static_cast<long long>(c->F) * c->T * c->H * (c->D / 8);
-  const ll_status st = launch_scatter(c, q, reinterpret_cast<cudaStream_t>(stream));
-  if (st == LL_OK) c->p[layer] += c->F;
-  return st;
+  const ll_status r = launch_scatter(c, q, 1, st);
+  if (r == LL_OK) {
+    c->p[layer] += c->F;
+    if (cs != cudaStreamCaptureStatusNone) c->host_counters = false;
+  }
+  return r;
 }
 
 ll_status ll_kv_recache_write(ll_kv_cache *c, int layer, const void *k_new, const void *v_new, int first_frame,
@@ -349,24 +395,23 @@ ll_status ll_kv_recache_write(ll_kv_cache *c, int layer, const void *k_new, cons
   if (first_frame < 0 || num_frames < 1) return LL_ERR_INVALID_ARG;
   const int l0 = layer < 0 ? 0 : layer;
   const int nl = layer < 0 ? c->L : 1;
-  // every addressed layer must hold the same context (same counter) so that one
-  // launch can apply one logical->slot map
-  int s = 0, w = 0;
-  held(c, l0, &s, &w);
-  for (int l = l0; l < l0 + nl; ++l) {
-    if (c->p[l] != c->p[l0]) return LL_ERR_INVALID_ARG;
+  if (static_cast<long long>(first_frame) + num_frames > c->S + c->W) return LL_ERR_INVALID_ARG;
+  // every addressed layer must hold the frames addressed; each layer maps logical
+  // frames to slots with its own counter. While the host mirror is exact this is
+  // checked here; otherwise the kernel skips such a layer and flags ERR_RANGE.
+  if (c->host_counters) {
+    for (int l = l0; l < l0 + nl; ++l) {
+      int s = 0, w = 0;
+      held(c, l, &s, &w);
+      if (static_cast<long long>(first_frame) + num_frames > s + w) return LL_ERR_INVALID_ARG;
+    }
   }
-  if (static_cast<long long>(first_frame) + num_frames > s + w) return LL_ERR_INVALID_ARG;
   llk::ScatterParams q = scatter_base(c, k_new, v_new);
   q.mode = llk::SCATTER_RECACHE;
   q.layer0 = l0;
   q.n_frames = num_frames;
-  q.p = kernel_p(c, l0);
-  q.s = s;
-  q.w = w;
   q.first = first_frame;
-  q.total_vec = static_cast<long long>(nl) * num_frames * c->T * c->H * (c->D / 8);
-  return launch_scatter(c, q, reinterpret_cast<cudaStream_t>(stream));
+  return launch_scatter(c, q, nl, reinterpret_cast<cudaStream_t>(stream));
 }
 
 ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cur, ll_kv_cache *c, int layer,
@@ -375,8 +420,6 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out)) return LL_ERR_INVALID_ARG;
   if (out == q || out == k_cur || out == v_cur) return LL_ERR_INVALID_ARG;
   const int Tq = c->F * c->T;
-  int s = 0, w = 0;
-  held(c, layer, &s, &w);
   llk::AttnParams prm;
   std::memset(&prm, 0, sizeof(prm));
   if (!make_act_map(&prm.tm_q, q, Tq, c->H, c->D) || !make_act_map(&prm.tm_kcur, k_cur, Tq, c->H, c->D) ||
@@ -388,9 +431,12 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   prm.tm_cache = quantised ? c->tm_view : c->tm_cache;
   prm.out = static_cast<__nv_bfloat16 *>(out);
   prm.err = c->err;
+  prm.frames = c->frames + layer;   // the kernel derives the visible keys from p
+  prm.S = c->S;
+  prm.W = c->W;
+  prm.T = c->T;
   prm.H = c->H;
   prm.Tq = Tq;
-  prm.n_cache = (s + w) * c->T;
   prm.plane_k = quantised ? 0 : (layer * 2 + 0) * c->H;
   prm.plane_v = quantised ? c->H : (layer * 2 + 1) * c->H;
   prm.num_q_tiles = (Tq + 127) / 128;
@@ -398,7 +444,7 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   const int grid = prm.num_q_tiles * c->H;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (quantised) {
-    const ll_status ds = launch_dequant(c, layer, prm.n_cache, st);
+    const ll_status ds = launch_dequant(c, layer, st);
     if (ds != LL_OK) return ds;
   }
   return c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
@@ -488,7 +534,7 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
   const int Tq = static_cast<int>(tq);
 
   // 1) dequantise the held rows into the view; the rows the ragged last tile
-  //    also reads, [n_cache, min(slots, 128 * ceil(n_cache / 128))), are cleared
+  //    also reads, [n_cache, min(slots, kKeyTile * ceil(n_cache / kKeyTile))), are cleared
   //    so that they are finite (the array keeps the previous call's contents)
   if (n_cache > 0) {
     llk::DequantParams dq;
@@ -498,10 +544,13 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
     dq.H = heads;
     dq.D = head_dim;
     dq.slots = static_cast<int>(slots);
+    dq.frames = nullptr;
     dq.n_rows = n_cache;
+    dq.S = sink_frames;
+    dq.W = window_frames;
+    dq.T = tokens_per_frame;
     dq.plane0 = 0;
-    dq.total_vec = static_cast<long long>(2 * heads) * n_cache * (head_dim / 8);
-    long long blocks = (dq.total_vec + 255) / 256;
+    long long blocks = (static_cast<long long>(2 * heads) * n_cache * (head_dim / 8) + 255) / 256;
     const long long cap = static_cast<long long>(num_sms(dev)) * 8;
     if (blocks > cap) blocks = cap;
     if (kv_dtype == LL_KV_FP8_E4M3)
@@ -509,7 +558,7 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
     else
       llk::kv_dequant_kernel<llk::FMT_NVFP4><<<static_cast<int>(blocks), 256, 0, st>>>(dq);
     if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
-    long long tail_end = (static_cast<long long>(n_cache) + 127) / 128 * 128;
+    long long tail_end = (static_cast<long long>(n_cache) + kKeyTile - 1) / kKeyTile * kKeyTile;
     if (tail_end > slots) tail_end = slots;
     if (tail_end > n_cache) {
       const size_t row_b = static_cast<size_t>(head_dim) * 2;
@@ -526,7 +575,7 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
   if (!make_act_map(&prm.tm_q, q, Tq, heads, head_dim) || !make_act_map(&prm.tm_kcur, k_cur, Tq, heads, head_dim) ||
       !make_act_map(&prm.tm_vcur, v_cur, Tq, heads, head_dim) ||
       !make_map_3d(&prm.tm_cache, view, head_dim, slots, 2 * heads, static_cast<uint64_t>(head_dim) * 2,
-                   static_cast<uint64_t>(slots) * head_dim * 2, 64, 128, 1))
+                   static_cast<uint64_t>(slots) * head_dim * 2, 64, kKeyTile, 1))
     return LL_ERR_CUDA;
   prm.out = static_cast<__nv_bfloat16 *>(out);
   prm.err = nullptr;

@@ -9,13 +9,14 @@
 namespace llk {
 
 // ---------------------------------------------------------------------------
-// status word written by kernels when a bounded wait gives up
-// low byte = reason, next byte = kernel id
+// status word written by kernels (OR-ed flags, cleared only by the host):
+// low byte = reasons, next byte = kernels that reported them
 enum : unsigned {
-  ERR_WAIT_TIMEOUT = 1u,
+  ERR_WAIT_TIMEOUT = 1u,     // a bounded wait gave up
+  ERR_RANGE = 2u,            // a recache addressed frames the layer does not hold
   KID_ATTN = 1u << 8,
   KID_SCATTER = 2u << 8,
-  KID_SELFTEST = 3u << 8,
+  KID_SELFTEST = 4u << 8,
 };
 
 // A wait that is not satisfied after this many SM clocks (~1.1 s at 1.9 GHz)

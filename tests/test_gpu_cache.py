@@ -150,7 +150,7 @@ def test_invalid_recache_ranges_are_rejected():
         with pytest.raises(ll.LLError):          # nothing held yet
             ll.ll_kv_recache_write(cache, 0, buf, buf, 0, 1)
         ll.ll_kv_append(cache, 0, buf, buf)
-        with pytest.raises(ll.LLError):          # layers hold different contexts
+        with pytest.raises(ll.LLError):          # layer 1 holds nothing yet
             ll.ll_kv_recache_write(cache, -1, buf, buf, 0, 1)
         with pytest.raises(ll.LLError):          # past the held frames
             ll.ll_kv_recache_write(cache, 0, buf, buf, 2, 2)

@@ -26,7 +26,7 @@ def test_bounded_wait_reports_timeout_and_context_stays_usable():
         torch.cuda.synchronize()
         word = ll.ll_debug_status(cache, clear=True)
         assert word & 0xFF == 1                     # wait timed out
-        assert (word >> 8) & 0xFF == 3              # reported by the self-test kernel
+        assert (word >> 8) & 0xFF == 4              # reported by the self-test kernel
         assert ll.ll_debug_status(cache) == 0       # cleared
         hk, hv = [], []
         for c in range(3):
