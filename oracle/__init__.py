@@ -24,9 +24,12 @@ Parity pins (what each function is checked against, in tests/test_oracle_*.py):
               configuration (tests/golden/).
   cache_model a list/deque simulation of "sink frames + last W frames";
               recache equivalence; constant footprint.
+  multi-shot  reduction to the single-shot rule; a hand-derived two-shot
+              example (tests/golden/); the cache model's held frames against
+              the frame-classification definition; recache equivalence.
   quant       exhaustive code tables; ml_dtypes' round-to-nearest-even casts;
               hand-listed ties and saturation cases (tests/golden/).
 """
-from .attention import visible_key_frames, key_mask, sink_window_attention  # noqa: F401
+from .attention import visible_key_frames, key_mask, sink_window_attention, multishot_visible_frames  # noqa: F401
 from .cache_model import CacheModel  # noqa: F401
 from . import quant  # noqa: F401

@@ -57,6 +57,51 @@ def visible_key_frames(chunk: int, S: int, W: int, F: int) -> list[int]:
     return [f for f in range((chunk + 1) * F) if frame_visible(chunk * F, f, S, W, F)]
 
 
+def multishot_visible_frames(chunk: int, G: int, Ss: int, W: int, F: int, shots=()) -> list[int]:
+    """Frames whose keys the queries of `chunk` see when the video has several shots.
+
+    LongLive-2.0 explainer (wmrh.cn, sec. 16): a global-level sink that every
+    shot attends to (identity, style, long-term context) and a shot-level sink
+    that keeps the current shot's own early frames; the short recent window of
+    LongLive (dpshk.com sec. 五) stays. Readings where the page is silent:
+      * the global sink is the first G frames of the video;
+      * the shot sink of a shot is its first Ss frames that are not global-sink
+        frames; a new shot empties it (its old frames are no longer seen);
+      * every other frame is a window frame; the window is the last W window
+        frames before the chunk, across shots, counted from the last shot start
+        that asked to clear it;
+      * the chunk's own frames are fully visible.
+    shots: (start_chunk, clear_window) of every shot after the first, which
+    starts at chunk 0. With Ss = 0 and no shots this is visible_key_frames.
+    """
+    starts = sorted(shots)
+    assert all(0 < c for c, _ in starts)
+
+    def shot_start_frame(f):
+        b = 0
+        for c, _ in starts:
+            if c * F <= f:
+                b = c * F
+        return b
+
+    def is_shot_sink(f):
+        lo = max(shot_start_frame(f), G)
+        return f >= G and f - lo < Ss
+
+    first = chunk * F
+    cur_lo = max(shot_start_frame(first), G)
+    clear_from = 0
+    for c, clear in starts:
+        if c <= chunk and clear:
+            clear_from = c * F
+    global_sink = [f for f in range(min(G, first))]
+    shot_sink = [f for f in range(cur_lo, min(cur_lo + Ss, first))]
+    window_frames = [f for f in range(max(G, clear_from), first) if not is_shot_sink(f)]
+    window = window_frames[max(0, len(window_frames) - W):] if W > 0 else []
+    own = list(range(first, first + F))
+    return sorted(set(global_sink) | set(shot_sink) | set(window) | set(own))
+
+
 def key_mask(chunk: int, query_rows: np.ndarray, n_key_tokens: int, S: int, W: int, F: int, T: int) -> np.ndarray:
     """Explicit boolean mask [len(query_rows)][n_key_tokens].
 
@@ -77,7 +122,7 @@ def key_mask(chunk: int, query_rows: np.ndarray, n_key_tokens: int, S: int, W: i
 
 def sink_window_attention(q_bits: np.ndarray, k_hist_bits: np.ndarray, v_hist_bits: np.ndarray,
                           chunk: int, S: int, W: int, F: int, T: int,
-                          rows=None, row_block: int = 256) -> np.ndarray:
+                          rows=None, row_block: int = 256, visible_frames=None) -> np.ndarray:
     """Attention output of chunk `chunk` in fp64.
 
     q_bits       [F*T][H][D] bf16 bits, the chunk's queries
@@ -85,6 +130,8 @@ def sink_window_attention(q_bits: np.ndarray, k_hist_bits: np.ndarray, v_hist_bi
                  generated so far, in generation order, the current chunk's K last
     v_hist_bits  same for V
     rows         optional subset of query rows (token index in the chunk)
+    visible_frames  optional explicit set of visible frames (e.g. from
+                 multishot_visible_frames), used instead of the S/W rule
     returns      [len(rows)][H][D] float64
     """
     Tq, H, D = q_bits.shape
@@ -100,7 +147,12 @@ def sink_window_attention(q_bits: np.ndarray, k_hist_bits: np.ndarray, v_hist_bi
         for r0 in range(0, len(rows), row_block):
             rr = rows[r0:r0 + row_block]
             q = _bf16_to_f64(q_bits[rr, h, :])                      # [R][D]
-            mask = key_mask(chunk, rr, n_keys, S, W, F, T)          # [R][N]
+            if visible_frames is None:
+                mask = key_mask(chunk, rr, n_keys, S, W, F, T)      # [R][N]
+            else:
+                vis = np.zeros(n_keys // T, dtype=bool)
+                vis[list(visible_frames)] = True
+                mask = np.broadcast_to(vis[np.arange(n_keys) // T][None, :], (len(rr), n_keys))
             s = (q @ k.T) * scale
             s = np.where(mask, s, -np.inf)
             s = s - s.max(axis=1, keepdims=True)

@@ -27,6 +27,19 @@ Readings taken where the pages are silent (the library follows the same ones):
 * Inputs are token-major [tokens][H][D] bf16; the source of a recache is
   [layers'][n*T][H][D] with layers' = 1 for one layer, L for all layers.
 
+Several shots (LongLive-2.0 explainer, wmrh.cn, sec. 16: a global-level sink
+all shots attend to and a shot-level sink per shot). With Ss shot-sink frames
+the layout per plane becomes [(S+Ss+W)*T]: slots 0..S-1 global sink,
+S..S+Ss-1 shot sink, then the W-slot ring. Each appended frame goes to exactly
+one region, in order: f < S -> global slot f; else, while the current shot's
+sink holds fewer than Ss frames -> the next shot-sink slot; else -> the next
+ring slot, S + Ss + (ring count mod W) (later frames of a chunk overwrite
+earlier ones when W < F, so only the last W survive). shot_begin empties the
+shot sink (and, if asked, starts the window afresh). Held context, in logical
+order: global sink, shot sink (fill order), window (oldest to newest, at most
+the last W ring frames since the last window restart). With Ss = 0 and no
+shot_begin this is exactly the single-shot rule above.
+
 Stored formats: "bf16" raw bits; "fp8" E4M3 codes + one fp32 scale per
 (token, head) row; "nvfp4" packed E2M1 codes + one E4M3 scale per 16 values.
 Export of a layer = data of K, data of V, then (quantised formats) scales of K,
@@ -41,12 +54,14 @@ from . import quant
 
 class CacheModel:
     def __init__(self, layers: int, heads: int, head_dim: int, tokens_per_frame: int,
-                 frames_per_chunk: int, sink_frames: int, window_frames: int, kv_dtype: str = "bf16"):
+                 frames_per_chunk: int, sink_frames: int, window_frames: int, kv_dtype: str = "bf16",
+                 shot_sink_frames: int = 0):
         assert kv_dtype in ("bf16", "fp8", "nvfp4")
         self.L, self.H, self.D = layers, heads, head_dim
         self.T, self.F, self.S, self.W = tokens_per_frame, frames_per_chunk, sink_frames, window_frames
+        self.Ss = shot_sink_frames
         self.kv_dtype = kv_dtype
-        self.slots = (self.S + self.W) * self.T
+        self.slots = (self.S + self.Ss + self.W) * self.T
         shape = (layers, 2, heads, self.slots)
         if kv_dtype == "bf16":
             self.data = np.zeros(shape + (head_dim,), dtype=np.uint16)
@@ -57,31 +72,52 @@ class CacheModel:
         else:
             self.data = np.zeros(shape + (head_dim // 2,), dtype=np.uint8)
             self.scales = np.zeros(shape + (head_dim // 16,), dtype=np.uint8)
-        self.p = [0] * layers
+        self.p = [0] * layers              # frames appended
+        self.shot_fill = [0] * layers      # frames in the current shot's sink
+        self.ring_count = [0] * layers     # frames that went to the ring
+        self.ring_start = [0] * layers     # ring count at the last window restart
+        self.slot_frame = [dict() for _ in range(layers)]   # frame slot -> absolute frame it holds
 
     # -- slot rules ---------------------------------------------------------
-    def append_slot(self, f: int, p: int):
-        """Physical frame slot of absolute frame f appended in a chunk that starts at p, or None."""
+    def _route(self, layer: int, f: int):
+        """Frame slot of absolute frame f, appended next to `layer`, or None;
+        advances the shot-sink fill and the ring count."""
         if f < self.S:
             return f
-        if self.W > 0 and f >= p + self.F - self.W:
-            return self.S + (f - self.S) % self.W
-        return None
+        if self.shot_fill[layer] < self.Ss:
+            slot = self.S + self.shot_fill[layer]
+            self.shot_fill[layer] += 1
+            return slot
+        idx = self.ring_count[layer]
+        self.ring_count[layer] += 1
+        if self.W == 0:
+            return None
+        return self.S + self.Ss + idx % self.W
 
     def held(self, layer: int):
-        p = self.p[layer]
-        s = min(p, self.S)
-        w = min(self.W, max(0, p - self.S))
-        return s, w
+        """(global sink frames, window frames) held; see held3 for the shot sink."""
+        g, sf, w = self.held3(layer)
+        assert self.Ss == 0
+        return g, w
+
+    def held3(self, layer: int):
+        g = min(self.p[layer], self.S)
+        sf = self.shot_fill[layer]
+        w = min(self.W, self.ring_count[layer] - self.ring_start[layer])
+        return g, sf, w
+
+    def n_held(self, layer: int) -> int:
+        return sum(self.held3(layer))
 
     def logical_slot(self, layer: int, k: int) -> int:
-        p = self.p[layer]
-        s, w = self.held(layer)
-        assert 0 <= k < s + w
-        if k < s:
+        g, sf, w = self.held3(layer)
+        assert 0 <= k < g + sf + w
+        if k < g:
             return k
-        a = p - w + (k - s)
-        return self.S + (a - self.S) % self.W
+        if k < g + sf:
+            return self.S + (k - g)
+        idx = self.ring_count[layer] - w + (k - g - sf)
+        return self.S + self.Ss + idx % self.W
 
     # -- writes -------------------------------------------------------------
     def _store_frame(self, layer: int, kv: int, slot: int, src_bits: np.ndarray):
@@ -103,20 +139,27 @@ class CacheModel:
         """k_cur, v_cur: [F*T][H][D] bf16 bits of the chunk just generated."""
         p = self.p[layer]
         for fi in range(self.F):
-            slot = self.append_slot(p + fi, p)
+            slot = self._route(layer, p + fi)
             if slot is None:
                 continue
             tok = slice(fi * self.T, (fi + 1) * self.T)
             self._store_frame(layer, 0, slot, k_cur[tok])
             self._store_frame(layer, 1, slot, v_cur[tok])
+            self.slot_frame[layer][slot] = p + fi
         self.p[layer] = p + self.F
+
+    def shot_begin(self, layer: int, clear_window: bool = False):
+        """A new shot starts with the next appended frame (layer -1 = all layers)."""
+        for l in (range(self.L) if layer < 0 else [layer]):
+            self.shot_fill[l] = 0
+            if clear_window:
+                self.ring_start[l] = self.ring_count[l]
 
     def recache_write(self, layer: int, k_new: np.ndarray, v_new: np.ndarray, first: int, num: int):
         """layer -1 = all layers. k_new/v_new: [layers'][num*T][H][D] bf16 bits."""
         layers = range(self.L) if layer < 0 else [layer]
         for li, l in enumerate(layers):
-            s, w = self.held(l)
-            assert 0 <= first and first + num <= s + w
+            assert 0 <= first and first + num <= self.n_held(l)
             for fi in range(num):
                 slot = self.logical_slot(l, first + fi)
                 tok = slice(fi * self.T, (fi + 1) * self.T)
@@ -138,10 +181,9 @@ class CacheModel:
 
     def logical_view(self, layer: int, kv: int) -> np.ndarray:
         """Stored rows of the held context in logical order, token-major:
-        [(s+w)*T][H][...] (bf16 bits, or codes for the quantised formats)."""
-        s, w = self.held(layer)
+        [n_held*T][H][...] (bf16 bits, or codes for the quantised formats)."""
         frames = []
-        for k in range(s + w):
+        for k in range(self.n_held(layer)):
             slot = self.logical_slot(layer, k)
             frames.append(np.transpose(self.data[layer, kv, :, slot * self.T:(slot + 1) * self.T], (1, 0, 2)))
         if not frames:
@@ -149,16 +191,13 @@ class CacheModel:
         return np.concatenate(frames, axis=0)
 
     def held_frames(self, layer: int, kv: int) -> dict:
-        """Held context as {absolute frame number: fp64 values [T][H][D]}: the sink
-        frames 0..s-1 and the window frames p-w..p-1, each dequantised exactly
-        (bf16 bits, or E4M3 code x fp32 row scale, or E2M1 code x E4M3 block
-        scale, in fp64)."""
-        p = self.p[layer]
-        s, w = self.held(layer)
+        """Held context as {absolute frame number: fp64 values [T][H][D]}, each
+        frame dequantised exactly (bf16 bits, or E4M3 code x fp32 row scale, or
+        E2M1 code x E4M3 block scale, in fp64)."""
         out = {}
-        for k in range(s + w):
-            frame = k if k < s else p - w + (k - s)
+        for k in range(self.n_held(layer)):
             slot = self.logical_slot(layer, k)
+            frame = self.slot_frame[layer][slot]
             sl = slice(slot * self.T, (slot + 1) * self.T)
             if self.kv_dtype == "bf16":
                 rows = (self.data[layer, kv, :, sl].astype(np.uint32) << np.uint32(16)).view(np.float32) \
