@@ -482,6 +482,36 @@ def run_ours(args, world, rank, local):
         res["speedup"] = res["full_causal"]["attn_ms_total"] / res["sink_window"]["attn_ms_total"]
         sweep["full_causal_vs_sink_window_40_chunks"] = res
 
+    # ---- several shots (global sink + per-shot sink + window), same 12-frame
+    # budget as the headline stack: global 3 + shot 3 + window 6. A shot starts
+    # every 8 chunks; every second start also restarts the window, so the
+    # window's ring range wraps and the visible keys come in up to 3 ranges.
+    multishot = None
+    if not args.no_multishot:
+        Gm, Ssm, Wm, n_chunks, every = S, 3, W - 3, 40, 8
+        mc = ll.ll_kv_cache_create_multishot(L, H, D, T, F, Gm, Ssm, Wm)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_chunks)]
+        flop = []
+        for c in range(n_chunks):
+            if c > 0 and c % every == 0:
+                ll.ll_kv_shot_begin(mc, -1, c % (2 * every) == 0, stream)
+            g_h, sf_h, w_h = ll.ll_kv_cache_held(mc, 0)
+            flop.append(L * 4.0 * TQ * (g_h + sf_h + w_h + F) * T * D * H)
+            evs[c][0].record(stream)
+            for l in range(L):
+                ll.ll_attn_sink_window(qs[l], ks[l], vs[l], mc, l, outs[l], stream)
+                ll.ll_kv_append(mc, l, ks[l], vs[l], stream)
+            evs[c][1].record(stream)
+        torch.cuda.synchronize(dev)
+        ms = [a.elapsed_time(b) for a, b in evs]
+        steady = range(4, n_chunks)        # the global sink and first shot sink are full from chunk 2 on
+        multishot = {"global_sink_frames": Gm, "shot_sink_frames": Ssm, "window_frames": Wm,
+                     "chunks": n_chunks, "shot_every_chunks": every, "window_restart_every_chunks": 2 * every,
+                     "ms_per_step": statistics.mean(ms[c] for c in steady),
+                     "tflops": sum(flop[c] for c in steady) / (sum(ms[c] for c in steady) * 1e-3) / 1e12,
+                     "cache_gb": ll.ll_kv_cache_info(mc, 0)[1] / 1e9, "device_status": ll.ll_debug_status(mc)}
+        mc.close()
+
     # ---- CPU oracle baseline (rank 0, single GPU only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -519,6 +549,7 @@ def run_ours(args, world, rank, local):
         "cpu_baseline": cpu,
         "quantised_cache": quant or None,
         "long_rollout": sweep,
+        "multishot": multishot,
         "device_status": status,
     }
     if rank == 0:
@@ -537,6 +568,7 @@ def main():
     ap.add_argument("--quant-steps", type=int, default=10)
     ap.add_argument("--no-sweep", action="store_true", help="skip the window sweep / full-causal leg")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
+    ap.add_argument("--no-multishot", action="store_true", help="skip the multi-shot cache leg")
     ap.add_argument("--layers", type=int, default=30, help="stack depth (30 = the Wan-1.3B stack)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="CPU seconds the reference arm spends in total (bounded sample per step)")

@@ -96,13 +96,40 @@ LL_API ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tok
                              int frames_per_chunk, int sink_frames, int window_frames,
                              ll_kv_dtype kv_dtype, ll_kv_cache **out);
 
+/* ll_kv_cache_create_multishot - a cache for videos of several shots.
+ *   LongLive-2.0 explainer (wmrh.cn), sec. 16: a global-level sink that every
+ *   shot attends to and a shot-level sink for the current shot. Per layer and
+ *   K/V plane the layout is [H][(G+Ss+W)*T][D]: slots 0..G-1 global sink (the
+ *   first G frames of the video), slots G..G+Ss-1 the current shot's sink (its
+ *   first Ss frames that are not global-sink frames), then a W-slot ring for
+ *   all other frames; the window is the ring's last W frames (since the last
+ *   window restart, see ll_kv_shot_begin). Each frame is stored in exactly one
+ *   region, so no key is attended twice. shot_sink_frames = 0 gives exactly
+ *   the single-shot cache of ll_kv_cache_create (which calls this with 0).
+ *   Other arguments, limits and errors as for ll_kv_cache_create, with
+ *   G + Ss + W >= 1 and (G+Ss+W)*T < 2^31.                                   */
+LL_API ll_status ll_kv_cache_create_multishot(int layers, int heads, int head_dim, int tokens_per_frame,
+                                              int frames_per_chunk, int global_sink_frames, int shot_sink_frames,
+                                              int window_frames, ll_kv_dtype kv_dtype, ll_kv_cache **out);
+
+/* ll_kv_shot_begin - a new shot starts with the next appended chunk.
+ *   layer: 0..L-1, or -1 for all layers. Empties the shot sink (its frames are
+ *   no longer attended; the next Ss non-global frames refill it). With
+ *   clear_window != 0 the window restarts too: it holds only frames appended
+ *   after this call. Enqueued on `stream` (a one-block kernel), so it is ordered
+ *   with the appends and can be recorded in a graph. A no-op on the shot sink
+ *   of a cache made with shot_sink_frames = 0. Pages: wmrh.cn sec. 16.          */
+LL_API ll_status ll_kv_shot_begin(ll_kv_cache *cache, int layer, int clear_window, ll_stream_t stream);
+
 /* ll_kv_append - store the chunk just generated in layer `layer` and evict.
  *   k_cur, v_cur: [F*T][H][D] bf16 device pointers (the chunk's K and V).
  *   Frame f = p..p+F-1 (p = frames appended to this layer so far) goes to slot
  *   f if f < S; otherwise, if f >= p+F-W, to ring slot S + ((f-S) mod W),
  *   overwriting (evicting) the oldest window frame; other frames (only when
- *   W < F) are not stored. Quantised caches quantise here. Then p += F, on
- *   the device, at the end of the launch (p is read from device memory).
+ *   W < F) are not stored. For a multi-shot cache, a non-global frame goes to
+ *   the current shot's sink while it has room, else to the next ring slot.
+ *   Quantised caches quantise here. Then p += F, on the device, at the end of
+ *   the launch (the counters are read from device memory).
  *   An append enqueued inside a stream capture ends the host's knowledge of
  *   p (see ll_kv_cache_info and ll_kv_recache_write).
  *   Pages: dpshk.com sec. 五/六; techwalker.com sec. 六.                    */
@@ -114,9 +141,11 @@ LL_API ll_status ll_kv_append(ll_kv_cache *cache, int layer, const void *k_cur, 
  *   k_new, v_new: [L'][num_frames*T][H][D] bf16 device pointers, L' = 1 for a
  *   single layer or L for all layers; frame i of the source replaces logical
  *   frame first_frame+i of the held context, whose logical order is: sink
- *   frames 0..s-1, then window frames oldest to newest (s = min(p,S),
- *   w = min(W, max(0, p-S)), p the layer's own counter). Requires
- *   0 <= first_frame, num_frames >= 1, first_frame + num_frames <= S + W
+ *   frames 0..s-1, then (multi-shot caches) the current shot's sink frames in
+ *   fill order, then window frames oldest to newest (s = min(p,S),
+ *   w = min(W, max(0, p-S)) for a single-shot cache, p the layer's own
+ *   counter; ll_kv_cache_held gives the counts). Requires
+ *   0 <= first_frame, num_frames >= 1, first_frame + num_frames <= S + Ss + W
  *   (else LL_ERR_INVALID_ARG) and <= s + w of every addressed layer: checked
  *   by the host (LL_ERR_INVALID_ARG) while it knows p; after a captured
  *   append, by the kernel, which then writes nothing to such a layer and sets
@@ -133,7 +162,8 @@ LL_API ll_status ll_kv_recache_write(ll_kv_cache *cache, int layer, const void *
  *   out: [F*T][H][D] bf16 device pointer, written. out may not alias inputs.
  *   For each head: out = softmax(q K^T / sqrt(D)) V over the keys of
  *   cache slots [0, s*T) (sink), [S*T, (S+w)*T) (window; held frames in any
- *   ring order, softmax is order-free) and the chunk's own k_cur/v_cur
+ *   ring order, softmax is order-free) - for a multi-shot cache the global
+ *   sink, the current shot's sink and the window - and the chunk's own k_cur/v_cur
  *   (all Tq of them, no mask inside the chunk). s, w as for recache, taken
  *   from the layer's frame counter at call time: call it BEFORE ll_kv_append
  *   of the same chunk. bf16 operands, fp32 accumulation and softmax, the
@@ -162,6 +192,13 @@ LL_API const char *ll_status_string(ll_status status);
  * after a device-wide synchronisation (do not call it while capturing).     */
 LL_API ll_status ll_kv_cache_info(const ll_kv_cache *cache, int layer, long long *frames_seen,
                            size_t *device_bytes);
+
+/* Frames of `layer` held now: global sink, current shot sink, window. Read
+ * from the host's mirror, or, once an append or shot start has been enqueued
+ * inside a stream capture, from the device after a device-wide
+ * synchronisation (do not call it while capturing). Any output may be NULL.   */
+LL_API ll_status ll_kv_cache_held(const ll_kv_cache *cache, int layer, int *global_frames, int *shot_frames,
+                                  int *window_frames);
 
 /* Number of device allocations the library currently holds (all caches).
  * Constant between create and destroy: the footprint check of a rollout.   */

@@ -41,6 +41,9 @@ _sig = {
     "ll_debug_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint), _i, _vp]),
     "ll_attn_sink_window_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _ll, _vp, _vp]),
     "ll_debug_wait_selftest": (_i, [_vp, _vp]),
+    "ll_kv_cache_create_multishot": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
+    "ll_kv_shot_begin": (_i, [_vp, _i, _i, _vp]),
+    "ll_kv_cache_held": (_i, [_vp, _i, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -94,6 +97,7 @@ class KVCache:
         self.layers, self.heads, self.head_dim = layers, heads, head_dim
         self.tokens_per_frame, self.frames_per_chunk = tokens_per_frame, frames_per_chunk
         self.sink_frames, self.window_frames, self.kv_dtype = sink_frames, window_frames, kv_dtype
+        self.shot_sink_frames = 0
 
     @property
     def tq(self) -> int:
@@ -125,6 +129,32 @@ def ll_kv_cache_create(layers: int, heads: int, head_dim: int, tokens_per_frame:
                                    window_frames, dt, ctypes.byref(h)), "ll_kv_cache_create")
     return KVCache(h.value, layers, heads, head_dim, tokens_per_frame, frames_per_chunk, sink_frames,
                    window_frames, kv_dtype)
+
+
+def ll_kv_cache_create_multishot(layers: int, heads: int, head_dim: int, tokens_per_frame: int,
+                                 frames_per_chunk: int, global_sink_frames: int, shot_sink_frames: int,
+                                 window_frames: int, kv_dtype="bf16") -> KVCache:
+    dt = _DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    h = _vp()
+    _check(_lib.ll_kv_cache_create_multishot(layers, heads, head_dim, tokens_per_frame, frames_per_chunk,
+                                             global_sink_frames, shot_sink_frames, window_frames, dt,
+                                             ctypes.byref(h)), "ll_kv_cache_create_multishot")
+    cache = KVCache(h.value, layers, heads, head_dim, tokens_per_frame, frames_per_chunk, global_sink_frames,
+                    window_frames, kv_dtype)
+    cache.shot_sink_frames = shot_sink_frames
+    return cache
+
+
+def ll_kv_shot_begin(cache: KVCache, layer: int = -1, clear_window: bool = False, stream=None):
+    _check(_lib.ll_kv_shot_begin(cache.handle, layer, int(clear_window), _stream(stream)), "ll_kv_shot_begin")
+
+
+def ll_kv_cache_held(cache: KVCache, layer: int = 0):
+    """(global-sink, shot-sink, window) frames the layer holds now."""
+    g, sf, w = _i(), _i(), _i()
+    _check(_lib.ll_kv_cache_held(cache.handle, layer, ctypes.byref(g), ctypes.byref(sf), ctypes.byref(w)),
+           "ll_kv_cache_held")
+    return g.value, sf.value, w.value
 
 
 def ll_kv_append(cache: KVCache, layer: int, k_cur, v_cur, stream=None):

@@ -2,20 +2,21 @@
 //
 // Computes, per head h and query row i of the current chunk,
 //   out[i,h,:] = softmax_j( q[i,h,:] . k_j / sqrt(D) ) v_j
-// over the keys j of cache slots [0, n_cache) of layer l (sink frames followed
-// by the held window frames; the two are one contiguous slot range because the
-// window only holds frames once all S sink slots are filled) and the chunk's
-// own k_cur/v_cur (Tq keys, no mask inside the chunk). The key set follows the
+// over the keys j of the visible cache slots of layer l and the chunk's own
+// k_cur/v_cur (Tq keys, no mask inside the chunk). The key set follows the
 // LongLive pages: KV cache = sink frames + recent window (dpshk.com LongLive
-// explainer, sec. 五 and 六); own chunk visible, future invisible (LongLive-2.0
-// explainer, wmrh.cn, sec. 6).
+// explainer, sec. 五 and 六); with several shots, a global sink plus the
+// current shot's sink (LongLive-2.0 explainer, wmrh.cn, sec. 16); own chunk
+// visible, future invisible (wmrh.cn sec. 6). The visible cache slots form at
+// most three row ranges (cache_layout.cuh); in a single-shot rollout they are
+// the one range [0, (s + w) T).
 //
 // Work unit: one 128-row query tile of one head (one CTA). The key range is cut
 // into 128-key tiles; even tiles go to softmax warpgroup 0, odd tiles to
 // warpgroup 1 (split-KV inside the CTA), each with its own S and O accumulators
 // in tensor memory; the two partial results are merged with their row maxima
 // and sums in the epilogue. Tiles past the valid keys are never visited; only
-// the last tile of each segment masks its tail columns.
+// the last tile of each key range masks its tail columns.
 //
 // Roles (384 threads, three warpgroups):
 //   warps 0-3  softmax warpgroup 0 (thread t owns query row t = TMEM lane t)
@@ -35,6 +36,7 @@
 #pragma once
 #include <cuda_bf16.h>
 
+#include "cache_layout.cuh"
 #include "sm100_ptx.cuh"
 
 namespace llk {
@@ -46,11 +48,11 @@ struct AttnParams {
   CUtensorMap tm_cache;  // (D, slots, L*2*H) bf16, box (64, 128, 1)
   __nv_bfloat16 *out;    // [Tq][H][D]
   unsigned *err;         // status word (see sm100_ptx.cuh)
-  const long long *frames;  // this layer's device frame counter p, or null: then n_cache is used
+  const LayerCtr *ctr;   // this layer's counters (device), or null: then slots [0, n_cache) are visible
   int H;
   int Tq;
-  int n_cache;           // visible cache keys when frames is null: slots [0, n_cache)
-  int S, W, T;           // sink frames, window frames, tokens per frame (with frames)
+  int n_cache;           // visible cache keys when ctr is null
+  int G, Ss, W, T;       // global sink, shot sink, window frames; tokens per frame (with ctr)
   int plane_k;           // (l*2 + 0) * H : plane of head 0 of this layer's K
   int plane_v;           // (l*2 + 1) * H
   int num_q_tiles;
@@ -74,10 +76,11 @@ struct AttnCfg {
   //           s_full[2], p_full[2], o_full[2], mma_done
   static constexpr int NBAR = 1 + 4 * NST + 7;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // tmem base, abort flag, tile counts
+  static constexpr int OFF_RANGES = OFF_MISC + 32;          // the visible key ranges (KeyRanges)
   // m[2][128], l[2][128] of the epilogue merge reuse the Q tile: by then every
   // MMA (all of which read Q before the last PV) has completed
   static constexpr int OFF_STATS = OFF_Q;
-  static constexpr int SMEM_BYTES = OFF_MISC + 32;
+  static constexpr int SMEM_BYTES = OFF_RANGES + 64;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;      // slack for 1024-byte alignment
   static constexpr int THREADS = 384;   // 3 warpgroups; warps 10-11 idle
   // registers: launched with 384 x 168 = 64512; the producer/MMA warpgroup drops
@@ -97,20 +100,50 @@ struct AttnCfg {
 // FMA-pipe polynomials balances the two pipes.
 constexpr unsigned kPolyPairs = 0x88u;
 
-// Visible cache keys: (s + w) * T with s = min(p, S), w = min(W, max(0, p - S)),
-// p read from the layer's device counter (advanced by the append kernel), so
-// the same launch is right for any p, as when a captured graph is replayed.
-__device__ __forceinline__ int visible_cache_keys(const AttnParams &prm) {
-  if (!prm.frames) return prm.n_cache;
-  const long long p = __ldcg(prm.frames);
-  const long long s = p < prm.S ? p : prm.S;
-  long long w = p - prm.S;
-  w = w < 0 ? 0 : (w > prm.W ? prm.W : w);
-  return static_cast<int>((s + w) * prm.T);
+// The visible cache keys as up to three row ranges of the layer's planes, and
+// their 128-key tiles: ranges are read from the layer's device counters
+// (advanced by the append kernel), so one launch is right for any state, as
+// when a captured graph is replayed.
+struct KeyRanges {
+  int r0, n0, r1, n1, r2, n2;  // first row and row count of each range
+  int t1, t2, nc;              // first tile of ranges 1 and 2; cache tiles in all
+};
+
+__device__ __forceinline__ KeyRanges visible_key_ranges(const AttnParams &prm) {
+  KeyRanges k = {0, prm.n_cache, 0, 0, 0, 0, 0, 0, 0};
+  if (prm.ctr) {
+    const long long ring_count = __ldcg(&prm.ctr->ring_count);
+    const HeldFrames hf = held_frames(__ldcg(&prm.ctr->p), __ldcg(&prm.ctr->shot_fill), ring_count,
+                                      __ldcg(&prm.ctr->ring_start), prm.G, prm.W);
+    const FrameRanges fr = visible_ranges(hf, ring_count, prm.G, prm.Ss, prm.W);
+    k.r0 = fr.start[0] * prm.T;
+    k.n0 = fr.len[0] * prm.T;
+    k.r1 = fr.start[1] * prm.T;
+    k.n1 = fr.len[1] * prm.T;
+    k.r2 = fr.start[2] * prm.T;
+    k.n2 = fr.len[2] * prm.T;
+  }
+  k.t1 = (k.n0 + 127) / 128;
+  k.t2 = k.t1 + (k.n1 + 127) / 128;
+  k.nc = k.t2 + (k.n2 + 127) / 128;
+  return k;
 }
 
-__device__ __forceinline__ int tile_valid(int j, int nc, int n_cache, int Tq) {
-  if (j < nc) return min(128, n_cache - j * 128);
+// The ranges live in shared memory (written once by thread 0) and are read
+// where needed, so that they hold no registers across the tile loops.
+// first cache row of cache tile j (j < nc)
+__device__ __forceinline__ int cache_tile_row(const volatile KeyRanges *k, int j) {
+  if (j < k->t1) return k->r0 + j * 128;
+  if (j < k->t2) return k->r1 + (j - k->t1) * 128;
+  return k->r2 + (j - k->t2) * 128;
+}
+
+// valid keys of tile j: cache tiles, then the own chunk's tiles
+__device__ __forceinline__ int tile_valid(const volatile KeyRanges *k, int j, int Tq) {
+  const int t1 = k->t1, t2 = k->t2, nc = k->nc;
+  if (j < t1) return min(128, k->n0 - j * 128);
+  if (j < t2) return min(128, k->n1 - (j - t1) * 128);
+  if (j < nc) return min(128, k->n2 - (j - t2) * 128);
   return min(128, Tq - (j - nc) * 128);
 }
 
@@ -142,12 +175,13 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
   const int unit = blockIdx.x;
   const int h = unit / prm.num_q_tiles;
   const int q0 = (unit % prm.num_q_tiles) * C::BM;
-  const int n_cache = visible_cache_keys(prm);
-  const int nc = (n_cache + C::BN - 1) / C::BN;
+  volatile KeyRanges *kr = reinterpret_cast<volatile KeyRanges *>(smem + C::OFF_RANGES);
   const int nown = (prm.Tq + C::BN - 1) / C::BN;
-  const int n_tiles = nc + nown;
 
   if (threadIdx.x == 0) {
+    const KeyRanges k = visible_key_ranges(prm);
+    kr->r0 = k.r0; kr->n0 = k.n0; kr->r1 = k.r1; kr->n1 = k.n1; kr->r2 = k.r2; kr->n2 = k.n2;
+    kr->t1 = k.t1; kr->t2 = k.t2; kr->nc = k.nc;
     mbar_init(q_full, 1);
     for (int s = 0; s < C::NST; ++s) {
       mbar_init(k_full + s, 1);
@@ -178,6 +212,8 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_smem;
+  const int nc = kr->nc;
+  const int n_tiles = nc + nown;
   // column bases: S_g = tmem + 128 g, O_g = tmem + 256 + D g
 #define TM_S(g) (tmem + 128u * static_cast<uint32_t>(g))
 #define TM_O(g) (tmem + 256u + static_cast<uint32_t>(D) * static_cast<uint32_t>(g))
@@ -206,7 +242,7 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
         mbar_arrive_expect_tx(k_full + st, C::TILE_BYTES);
         if (j < nc) {
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d(sk + b * C::BOX_BYTES, &prm.tm_cache, k_full + st, b * 64, j * C::BN, prm.plane_k + h);
+            tma_load_3d(sk + b * C::BOX_BYTES, &prm.tm_cache, k_full + st, b * 64, cache_tile_row(kr, j), prm.plane_k + h);
         } else {
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_3d(sk + b * C::BOX_BYTES, &prm.tm_kcur, k_full + st, b * 64, h, (j - nc) * C::BN);
@@ -219,7 +255,7 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
         mbar_arrive_expect_tx(v_full + st, C::TILE_BYTES);
         if (j < nc) {
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d(sv + b * C::BOX_BYTES, &prm.tm_cache, v_full + st, b * 64, j * C::BN, prm.plane_v + h);
+            tma_load_3d(sv + b * C::BOX_BYTES, &prm.tm_cache, v_full + st, b * 64, cache_tile_row(kr, j), prm.plane_v + h);
         } else {
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_3d(sv + b * C::BOX_BYTES, &prm.tm_vcur, v_full + st, b * 64, h, (j - nc) * C::BN);
@@ -314,6 +350,8 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
     int it = 0;
     bool ok = true;
     for (int j = g; j < n_tiles; j += 2, ++it) {
+      // the tile's valid keys, read from shared memory while S is still computed
+      const int valid = tile_valid(kr, j, prm.Tq);
       // wait results are made warp-uniform: a warp never splits across the
       // .sync.aligned tensor-memory instructions that follow
       if (!__all_sync(0xffffffffu, mbar_wait(s_full + g, it & 1, abort_flag, prm.err, KID_ATTN))) {
@@ -327,7 +365,6 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
       uint32_t sr[128];
       tmem_ld64(TM_S(g) + lane_off, sr);
       tmem_ld64(TM_S(g) + lane_off + 64, sr + 64);
-      const int valid = tile_valid(j, nc, n_cache, prm.Tq);
       if (valid < 128) {
 #pragma unroll
         for (int e = 0; e < 128; ++e)

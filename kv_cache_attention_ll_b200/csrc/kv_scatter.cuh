@@ -3,12 +3,14 @@
 // Both operations copy whole frames of token-major K/V ([tokens][H][D] bf16, as
 // a QKV projection emits them) into the head-major cache planes
 // ([plane][slots][D], plane = (layer*2 + kv)*H + head), frame f of the source
-// landing in frame slot `slot_of(f)`:
+// landing in the frame slot that cache_layout.cuh assigns:
 //   append  (LongLive explainer, dpshk.com, sec. 五/六: sink kept, oldest window
-//            frame evicted): f < S -> f; f >= p+F-W -> S + ((f-S) mod W); else skip
+//            frame evicted; LongLive-2.0 explainer, wmrh.cn, sec. 16: shot sink):
+//            global sink, else the current shot's sink while it has room, else
+//            the next ring slot (append_slot)
 //   recache (dpshk.com sec. 三.5; techwalker.com LONGLIVE article sec. 六): logical
-//            frame k of the held context -> k if k < s, else the ring slot of
-//            absolute frame p - w + (k - s).
+//            frame k of the held context (global sink, shot sink, window) to its
+//            slot (logical_slot)
 // Grid: blockIdx.x = one (source layer, source frame) pair, blockIdx.y strides
 // over that frame's T*H*D/8 16-byte vectors. Everything that depends on the
 // layer's frame counter (the destination slot, or that nothing is stored) is
@@ -23,6 +25,7 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "cache_layout.cuh"
 #include "sm100_ptx.cuh"
 
 namespace llk {
@@ -40,35 +43,13 @@ struct ScatterParams {
   int layer0;                // first destination layer
   int n_frames;              // frames per source layer
   int mode;                  // ScatterMode
-  int S, W, F;               // cache geometry
+  int G, Ss, W, F;           // cache geometry: global sink, shot sink, window, chunk frames
   int first;                 // recache: first logical frame
-  long long *frames;         // per-layer frame counters p (device); append advances its layer's by F
-  unsigned *done;            // per-layer count of finished append blocks (zero between launches)
+  LayerCtr *ctr;             // per-layer counters (device); append advances its layer's
+  unsigned *done;            // per-layer count of finished append blocks (zero between launches),
+                             // kept away from the counters that every block reads
   unsigned *err;             // status word: recache beyond the held frames is flagged there
 };
-
-// Only whether p < S and the ring position (p - S) mod W matter once p >= S + W,
-// so very long rollouts fold into int range without changing any slot.
-__device__ __forceinline__ int fold_frames(long long p, int S, int W) {
-  if (p <= (1ll << 30)) return static_cast<int>(p);
-  if (W == 0) return S + W;
-  return S + W + static_cast<int>((p - S) % W);
-}
-
-// Destination frame slot of source frame fi, or -1 when it is not stored.
-// p: folded counter of the layer; s, w: its held sink and window frames.
-__device__ __forceinline__ int scatter_slot(const ScatterParams &q, int p, int s, int w, int fi) {
-  if (q.mode == SCATTER_APPEND) {
-    const int f = p + fi;
-    if (f < q.S) return f;
-    if (q.W > 0 && f >= p + q.F - q.W) return q.S + (f - q.S) % q.W;
-    return -1;
-  }
-  const int k = q.first + fi;
-  if (k < s) return k;
-  const int a = p - w + (k - s);
-  return q.S + (a - q.S) % q.W;
-}
 
 // 8 fp32 -> 8 E4M3 codes (round to nearest even, saturating), element 0 in byte 0
 __device__ __forceinline__ uint2 e4m3x8(const float (&y)[8]) {
@@ -120,15 +101,32 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
   const int li = blockIdx.x / q.n_frames;      // source layer
   const int fi = blockIdx.x % q.n_frames;      // source frame
   const int layer = q.layer0 + li;
-  // the layer's counter; every block reads it before its own completion count
-  // below, so the append's advance (by the last block) comes after all reads
-  const long long p_raw = __ldcg(q.frames + layer);
-  const int s_held = static_cast<int>(p_raw < q.S ? p_raw : q.S);
-  const int w_held = static_cast<int>(p_raw - q.S < 0 ? 0 : (p_raw - q.S > q.W ? q.W : p_raw - q.S));
-  // recache of frames the layer does not hold: nothing of that layer is written
-  const bool reject = q.mode == SCATTER_RECACHE && q.first + q.n_frames > s_held + w_held;
-  if (reject && fi == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(q.err, KID_SCATTER | ERR_RANGE);
-  const int slot = reject ? -1 : scatter_slot(q, fold_frames(p_raw, q.S, q.W), s_held, w_held, fi);
+  // the layer's counters, read once per block by thread 0 before the block's
+  // completion count below, so the append's advance (by the last block) comes
+  // after every block's read
+  __shared__ LayerCtr blk_ctr;
+  if (threadIdx.x == 0) {
+    const LayerCtr *lc = q.ctr + layer;
+    blk_ctr.p = __ldcg(&lc->p);
+    blk_ctr.ring_count = __ldcg(&lc->ring_count);
+    blk_ctr.ring_start = __ldcg(&lc->ring_start);
+    blk_ctr.shot_fill = __ldcg(&lc->shot_fill);
+  }
+  __syncthreads();
+  const long long p = blk_ctr.p;
+  const long long ring_count = blk_ctr.ring_count;
+  const long long ring_start = blk_ctr.ring_start;
+  const int shot_fill = blk_ctr.shot_fill;
+  int slot;
+  if (q.mode == SCATTER_APPEND) {
+    slot = append_slot(p, shot_fill, ring_count, q.G, q.Ss, q.W, q.F, fi);
+  } else {
+    const HeldFrames hf = held_frames(p, shot_fill, ring_count, ring_start, q.G, q.W);
+    // recache of frames the layer does not hold: nothing of that layer is written
+    const bool reject = q.first + q.n_frames > hf.g + hf.sf + hf.w;
+    if (reject && fi == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(q.err, KID_SCATTER | ERR_RANGE);
+    slot = reject ? -1 : logical_slot(hf, ring_count, q.G, q.Ss, q.W, q.first + fi);
+  }
   const long long src0 = static_cast<long long>(blockIdx.x) * q.frame_vec;   // first vector of the frame
   const int stride = gridDim.y * blockDim.x;
   // block-uniform trip count (slot is uniform too): every lane runs every
@@ -206,14 +204,20 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
     }
   }
   if (q.mode == SCATTER_APPEND) {
-    // the last block to finish advances the counter; every thread of every
-    // block read it above, before this barrier and its block's increment
+    // the last block to finish advances the counters; every block read them
+    // above, before its increment of the completion count
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
+      LayerCtr *c = q.ctr + q.layer0;
       const unsigned prev = atomicAdd(q.done + q.layer0, 1u);
       if (prev == gridDim.x * gridDim.y - 1) {
-        q.frames[q.layer0] = p_raw + q.F;
+        int fill;
+        long long rc;
+        append_advance(p, shot_fill, ring_count, q.G, q.Ss, q.F, &fill, &rc);
+        c->p = p + q.F;
+        c->shot_fill = fill;
+        c->ring_count = rc;
         q.done[q.layer0] = 0;
         __threadfence();
       }
@@ -243,9 +247,9 @@ struct DequantParams {
   const uint8_t *data;     // codes of all layers
   const uint8_t *scales;   // scales of all layers
   uint4 *view;             // [2H][slots][D] bf16
-  const long long *frames; // the layer's device frame counter, or null: then n_rows is used
+  const LayerCtr *ctr;     // the layer's counters, or null: then rows [0, n_rows) are converted
   int H, D, slots, n_rows;
-  int S, W, T;             // with frames: rows = (min(p,S) + min(W, max(0, p-S))) * T
+  int G, Ss, W, T;         // with ctr: the visible frame ranges of cache_layout.cuh are converted
   int plane0;              // first plane of the layer: layer * 2H
 };
 
@@ -269,20 +273,26 @@ template <int FMT>
 __global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) {
   const int vpr = q.D >> 3;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  int n_rows = q.n_rows;
-  if (q.frames) {
-    const long long p = __ldcg(q.frames);
-    const long long s = p < q.S ? p : q.S;
-    long long w = p - q.S;
-    w = w < 0 ? 0 : (w > q.W ? q.W : w);
-    n_rows = static_cast<int>((s + w) * q.T);
+  // visible rows as up to three slot-row ranges; rows are counted through them in order
+  int r0 = 0, n0 = q.n_rows, r1 = 0, n1 = 0, r2 = 0, n2 = 0;
+  if (q.ctr) {
+    const long long ring_count = __ldcg(&q.ctr->ring_count);
+    const HeldFrames hf = held_frames(__ldcg(&q.ctr->p), __ldcg(&q.ctr->shot_fill), ring_count,
+                                      __ldcg(&q.ctr->ring_start), q.G, q.W);
+    const FrameRanges fr = visible_ranges(hf, ring_count, q.G, q.Ss, q.W);
+    n0 = 0;
+    if (fr.n > 0) { r0 = fr.start[0] * q.T; n0 = fr.len[0] * q.T; }
+    if (fr.n > 1) { r1 = fr.start[1] * q.T; n1 = fr.len[1] * q.T; }
+    if (fr.n > 2) { r2 = fr.start[2] * q.T; n2 = fr.len[2] * q.T; }
   }
+  const int n_rows = n0 + n1 + n2;
   const long long total_vec = static_cast<long long>(2 * q.H) * n_rows * vpr;
   for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_vec; i += stride) {
     const int vec = static_cast<int>(i % vpr);
-    const long long pr = i / vpr;                       // (local plane, row)
-    const int row = static_cast<int>(pr % n_rows);
+    const long long pr = i / vpr;                       // (local plane, visible row)
+    const int vr = static_cast<int>(pr % n_rows);
     const int lp = static_cast<int>(pr / n_rows);       // 0 .. 2H-1
+    const int row = vr < n0 ? r0 + vr : (vr < n0 + n1 ? r1 + (vr - n0) : r2 + (vr - n0 - n1));
     const long long src_row = static_cast<long long>(q.plane0 + lp) * q.slots + row;
     uint32_t o[4];
     if constexpr (FMT == FMT_FP8) {

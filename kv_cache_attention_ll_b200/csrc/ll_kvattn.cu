@@ -27,9 +27,10 @@
 
 struct ll_kv_cache {
   int L, H, D, T, F, S, W;
+  int Ss;                     // shot-sink frames (0: a single-shot cache)
   ll_kv_dtype dtype;
   int device;
-  long long slots;            // (S+W)*T rows per plane
+  long long slots;            // (S+Ss+W)*T rows per plane
   uint8_t *base;              // the one allocation
   size_t bytes;               // its size
   uint8_t *data;              // [L][2][H][slots][row bytes]
@@ -37,10 +38,10 @@ struct ll_kv_cache {
   unsigned *err;              // device status word
   size_t data_plane_bytes;    // bytes of one plane's data
   size_t scale_plane_bytes;   // bytes of one plane's scales
-  std::vector<long long> p;   // host mirror of the frame counters (exact while host_counters)
-  bool host_counters;         // false once an append was enqueued inside a stream capture
-  long long *frames;          // device frame counters [L]
-  unsigned *done;             // device append-completion counts [L]
+  std::vector<llk::LayerCtr> hc;  // host mirror of the counters (exact while host_counters)
+  bool host_counters;         // false once an append or shot start was enqueued inside a stream capture
+  llk::LayerCtr *ctr;         // device counters [L]
+  unsigned *done;             // device append-completion counts [L] (own cache lines)
   CUtensorMap tm_cache;       // bf16 cache planes (D, slots, L*2*H)
   uint8_t *view;              // quantised caches: bf16 view of one layer [2H][slots][D]
   CUtensorMap tm_view;        // (D, slots, 2H) over the view
@@ -95,13 +96,21 @@ bool make_act_map(CUtensorMap *m, const void *p, int Tq, int H, int D) {
   return make_map_3d(m, p, D, H, Tq, static_cast<uint64_t>(D) * 2, static_cast<uint64_t>(H) * D * 2, 64, 1, kKeyTile);
 }
 
-void held(const ll_kv_cache *c, int layer, int *s, int *w) {
-  const long long p = c->p[layer];
-  *s = static_cast<int>(p < c->S ? p : c->S);
-  long long ww = p - c->S;
-  if (ww < 0) ww = 0;
-  if (ww > c->W) ww = c->W;
-  *w = static_cast<int>(ww);
+// held frames of a layer according to the host mirror
+llk::HeldFrames held(const ll_kv_cache *c, int layer) {
+  const llk::LayerCtr &h = c->hc[layer];
+  return llk::held_frames(h.p, h.shot_fill, h.ring_count, h.ring_start, c->S, c->W);
+}
+
+// the device counters of one layer (after a device-wide synchronisation)
+bool read_device_counters(const ll_kv_cache *c, int layer, llk::LayerCtr *out) {
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (cudaSetDevice(c->device) != cudaSuccess) return false;
+  const bool ok = cudaDeviceSynchronize() == cudaSuccess &&
+                  cudaMemcpy(out, c->ctr + layer, sizeof(*out), cudaMemcpyDeviceToHost) == cudaSuccess;
+  cudaSetDevice(prev);
+  return ok;
 }
 
 int num_sms(int device) {
@@ -137,9 +146,10 @@ ll_status launch_dequant(ll_kv_cache *c, int layer, cudaStream_t stream) {
   q.H = c->H;
   q.D = c->D;
   q.slots = static_cast<int>(c->slots);
-  q.frames = c->frames + layer;
+  q.ctr = c->ctr + layer;
   q.n_rows = 0;
-  q.S = c->S;
+  q.G = c->S;
+  q.Ss = c->Ss;
   q.W = c->W;
   q.T = c->T;
   q.plane0 = layer * 2 * c->H;
@@ -185,10 +195,11 @@ llk::ScatterParams scatter_base(const ll_kv_cache *c, const void *k, const void 
   q.T = c->T;
   q.frame_vec = c->T * c->H * (c->D / 8);
   q.slots = static_cast<int>(c->slots);
-  q.S = c->S;
+  q.G = c->S;
+  q.Ss = c->Ss;
   q.W = c->W;
   q.F = c->F;
-  q.frames = c->frames;
+  q.ctr = c->ctr;
   q.done = c->done;
   q.err = c->err;
   return q;
@@ -214,13 +225,23 @@ long long ll_allocation_count(void) { return g_alloc_count.load(); }
 
 ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per_frame, int frames_per_chunk,
                              int sink_frames, int window_frames, ll_kv_dtype kv_dtype, ll_kv_cache **out) {
+  return ll_kv_cache_create_multishot(layers, heads, head_dim, tokens_per_frame, frames_per_chunk, sink_frames, 0,
+                                      window_frames, kv_dtype, out);
+}
+
+ll_status ll_kv_cache_create_multishot(int layers, int heads, int head_dim, int tokens_per_frame,
+                                       int frames_per_chunk, int global_sink_frames, int shot_sink_frames,
+                                       int window_frames, ll_kv_dtype kv_dtype, ll_kv_cache **out) {
   if (!out) return LL_ERR_INVALID_ARG;
   *out = nullptr;
+  const int sink_frames = global_sink_frames;
   if (layers < 1 || heads < 1 || tokens_per_frame < 1 || frames_per_chunk < 1) return LL_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return LL_ERR_INVALID_ARG;
-  if (sink_frames < 0 || window_frames < 0 || sink_frames + window_frames < 1) return LL_ERR_INVALID_ARG;
+  if (sink_frames < 0 || shot_sink_frames < 0 || window_frames < 0) return LL_ERR_INVALID_ARG;
+  if (static_cast<long long>(sink_frames) + shot_sink_frames + window_frames < 1) return LL_ERR_INVALID_ARG;
   if (kv_dtype != LL_KV_BF16 && kv_dtype != LL_KV_FP8_E4M3 && kv_dtype != LL_KV_NVFP4) return LL_ERR_INVALID_ARG;
-  const long long slots = static_cast<long long>(sink_frames + window_frames) * tokens_per_frame;
+  const long long slots =
+      (static_cast<long long>(sink_frames) + shot_sink_frames + window_frames) * tokens_per_frame;
   const long long tq = static_cast<long long>(frames_per_chunk) * tokens_per_frame;
   if (slots >= (1ll << 31) || tq >= (1ll << 31)) return LL_ERR_INVALID_ARG;
   if (static_cast<long long>(tokens_per_frame) * heads * (head_dim / 8) >= (1ll << 30)) return LL_ERR_INVALID_ARG;
@@ -242,7 +263,8 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   // quantised caches also hold a bf16 view of one layer's K and V planes, the
   // input of the attention kernel after each call's dequantisation
   const size_t ctr_off = err_off + 256;
-  const size_t ctr_bytes = ((static_cast<size_t>(layers) * 12 + 255) / 256) * 256;   // counters, done counts
+  const size_t ctr_bytes = ((static_cast<size_t>(layers) * sizeof(llk::LayerCtr) + 255) / 256) * 256 +
+                           ((static_cast<size_t>(layers) * sizeof(unsigned) + 255) / 256) * 256;
   const size_t view_off = ctr_off + ctr_bytes;
   const size_t view_bytes =
       kv_dtype == LL_KV_BF16 ? 0 : static_cast<size_t>(2 * heads) * slots * head_dim * 2;
@@ -255,7 +277,8 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   if (!c) return LL_ERR_OOM;
   c->L = layers; c->H = heads; c->D = head_dim; c->T = tokens_per_frame; c->F = frames_per_chunk;
   c->S = sink_frames; c->W = window_frames; c->dtype = kv_dtype; c->device = dev; c->slots = slots;
-  c->p.assign(layers, 0);
+  c->Ss = shot_sink_frames;
+  c->hc.assign(layers, llk::LayerCtr{0, 0, 0, 0, 0});
   c->host_counters = true;
   c->data_plane_bytes = data_plane;
   c->scale_plane_bytes = scale_plane;
@@ -272,8 +295,9 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
   c->data = c->base;
   c->scales = scale_bytes ? c->base + scale_off : nullptr;
   c->err = reinterpret_cast<unsigned *>(c->base + err_off);
-  c->frames = reinterpret_cast<long long *>(c->base + ctr_off);
-  c->done = reinterpret_cast<unsigned *>(c->base + ctr_off + static_cast<size_t>(layers) * 8);
+  c->ctr = reinterpret_cast<llk::LayerCtr *>(c->base + ctr_off);
+  c->done = reinterpret_cast<unsigned *>(c->base + ctr_off +
+                                         ((static_cast<size_t>(layers) * sizeof(llk::LayerCtr) + 255) / 256) * 256);
   c->view = view_bytes ? c->base + view_off : nullptr;
   if (cudaMemset(mem, 0, total) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(mem);
@@ -316,19 +340,13 @@ ll_status ll_kv_cache_info(const ll_kv_cache *c, int layer, long long *frames_se
   if (!c || layer < 0 || layer >= c->L) return LL_ERR_INVALID_ARG;
   if (frames_seen) {
     if (c->host_counters) {
-      *frames_seen = c->p[layer];
+      *frames_seen = c->hc[layer].p;
     } else {
       // replays of captured appends have moved the device counter: wait for all
       // work on the device, then read it
-      int prev = 0;
-      cudaGetDevice(&prev);
-      if (cudaSetDevice(c->device) != cudaSuccess) return LL_ERR_CUDA;
-      long long v = 0;
-      const bool ok = cudaDeviceSynchronize() == cudaSuccess &&
-                      cudaMemcpy(&v, c->frames + layer, sizeof(v), cudaMemcpyDeviceToHost) == cudaSuccess;
-      cudaSetDevice(prev);
-      if (!ok) return LL_ERR_CUDA;
-      *frames_seen = v;
+      llk::LayerCtr d;
+      if (!read_device_counters(c, layer, &d)) return LL_ERR_CUDA;
+      *frames_seen = d.p;
     }
   }
   if (device_bytes) *device_bytes = c->bytes;
@@ -382,7 +400,13 @@ ll_status ll_kv_append(ll_kv_cache *c, int layer, const void *k_cur, const void 
   q.n_frames = c->F;
   const ll_status r = launch_scatter(c, q, 1, st);
   if (r == LL_OK) {
-    c->p[layer] += c->F;
+    llk::LayerCtr &h = c->hc[layer];
+    int fill = 0;
+    long long rc = 0;
+    llk::append_advance(h.p, h.shot_fill, h.ring_count, c->S, c->Ss, c->F, &fill, &rc);
+    h.p += c->F;
+    h.shot_fill = fill;
+    h.ring_count = rc;
     if (cs != cudaStreamCaptureStatusNone) c->host_counters = false;
   }
   return r;
@@ -395,15 +419,15 @@ ll_status ll_kv_recache_write(ll_kv_cache *c, int layer, const void *k_new, cons
   if (first_frame < 0 || num_frames < 1) return LL_ERR_INVALID_ARG;
   const int l0 = layer < 0 ? 0 : layer;
   const int nl = layer < 0 ? c->L : 1;
-  if (static_cast<long long>(first_frame) + num_frames > c->S + c->W) return LL_ERR_INVALID_ARG;
+  if (static_cast<long long>(first_frame) + num_frames > static_cast<long long>(c->S) + c->Ss + c->W)
+    return LL_ERR_INVALID_ARG;
   // every addressed layer must hold the frames addressed; each layer maps logical
   // frames to slots with its own counter. While the host mirror is exact this is
   // checked here; otherwise the kernel skips such a layer and flags ERR_RANGE.
   if (c->host_counters) {
     for (int l = l0; l < l0 + nl; ++l) {
-      int s = 0, w = 0;
-      held(c, l, &s, &w);
-      if (static_cast<long long>(first_frame) + num_frames > s + w) return LL_ERR_INVALID_ARG;
+      const llk::HeldFrames h = held(c, l);
+      if (static_cast<long long>(first_frame) + num_frames > h.g + h.sf + h.w) return LL_ERR_INVALID_ARG;
     }
   }
   llk::ScatterParams q = scatter_base(c, k_new, v_new);
@@ -431,8 +455,9 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   prm.tm_cache = quantised ? c->tm_view : c->tm_cache;
   prm.out = static_cast<__nv_bfloat16 *>(out);
   prm.err = c->err;
-  prm.frames = c->frames + layer;   // the kernel derives the visible keys from p
-  prm.S = c->S;
+  prm.ctr = c->ctr + layer;   // the kernel derives the visible keys from the layer's counters
+  prm.G = c->S;
+  prm.Ss = c->Ss;
   prm.W = c->W;
   prm.T = c->T;
   prm.H = c->H;
@@ -448,6 +473,57 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
     if (ds != LL_OK) return ds;
   }
   return c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
+}
+
+// ---------------------------------------------------------------------------
+// Shot start (several shots per video): empties the shot sink of the addressed
+// layers and, if asked, restarts their window. A kernel, so that it is ordered
+// with the appends on the stream and can be recorded in a graph.
+namespace llk {
+__global__ void shot_begin_kernel(LayerCtr *ctr, int l0, int nl, int clear_window) {
+  for (int i = threadIdx.x; i < nl; i += blockDim.x) {
+    LayerCtr *c = ctr + l0 + i;
+    c->shot_fill = 0;
+    if (clear_window) c->ring_start = c->ring_count;
+  }
+}
+}  // namespace llk
+
+extern "C" ll_status ll_kv_shot_begin(ll_kv_cache *c, int layer, int clear_window, ll_stream_t stream) {
+  if (!c || layer < -1 || layer >= c->L) return LL_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return LL_ERR_CUDA;
+  }
+  const int l0 = layer < 0 ? 0 : layer;
+  const int nl = layer < 0 ? c->L : 1;
+  llk::shot_begin_kernel<<<1, 256, 0, st>>>(c->ctr, l0, nl, clear_window ? 1 : 0);
+  if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
+  for (int l = l0; l < l0 + nl; ++l) {
+    c->hc[l].shot_fill = 0;
+    if (clear_window) c->hc[l].ring_start = c->hc[l].ring_count;
+  }
+  if (cs != cudaStreamCaptureStatusNone) c->host_counters = false;
+  return LL_OK;
+}
+
+extern "C" ll_status ll_kv_cache_held(const ll_kv_cache *c, int layer, int *global_frames, int *shot_frames,
+                                      int *window_frames) {
+  if (!c || layer < 0 || layer >= c->L) return LL_ERR_INVALID_ARG;
+  llk::HeldFrames h;
+  if (c->host_counters) {
+    h = held(c, layer);
+  } else {
+    llk::LayerCtr d;
+    if (!read_device_counters(c, layer, &d)) return LL_ERR_CUDA;
+    h = llk::held_frames(d.p, d.shot_fill, d.ring_count, d.ring_start, c->S, c->W);
+  }
+  if (global_frames) *global_frames = h.g;
+  if (shot_frames) *shot_frames = h.sf;
+  if (window_frames) *window_frames = h.w;
+  return LL_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -544,9 +620,10 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
     dq.H = heads;
     dq.D = head_dim;
     dq.slots = static_cast<int>(slots);
-    dq.frames = nullptr;
+    dq.ctr = nullptr;
     dq.n_rows = n_cache;
-    dq.S = sink_frames;
+    dq.G = sink_frames;
+    dq.Ss = 0;
     dq.W = window_frames;
     dq.T = tokens_per_frame;
     dq.plane0 = 0;
