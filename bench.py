@@ -47,8 +47,8 @@ ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out
 # ncu DRAM traffic of one attention launch at this shape and the kernel sources it
 # was taken with (profiles/attn_sink_window_wan1.3b.md); reported only while the
 # kernel is unchanged.
-ATTN_TRAFFIC = 165.80e6        # mean of the two captured launches (167.85 MB, 163.75 MB)
-ATTN_TRAFFIC_SRC_SHA = "9b360afb25ef9eca"
+ATTN_TRAFFIC = 167.0e6         # mean of the two captured launches (166.6 MB, 167.4 MB)
+ATTN_TRAFFIC_SRC_SHA = "8327bc4248d862ae"
 
 
 def _peaks():
