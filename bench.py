@@ -52,12 +52,16 @@ ATTN_TRAFFIC_SRC_SHA = "2cc1e069977cef9a"
 
 
 def _peaks():
+    """(bf16 burst TF/s, bf16 sustained TF/s, HBM GB/s, "measured" | "fallback").
+    The burst figure fits a kernel timed alone, the sustained one (seconds of
+    back-to-back GEMMs under the power cap) a kernel timed inside a long step."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
             p = json.load(fh)
-        return float(p["bf16_tflops"]), float(p["hbm_gbs"]), "measured"
+        return (float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                float(p["hbm_gbs"]), "measured")
     except Exception:
-        return 1590.0, 6650.0, "fallback"
+        return 1590.0, 1400.0, 6650.0, "fallback"
 
 
 def _kernel_sha() -> str:
@@ -234,7 +238,7 @@ def run_ours(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    peak_tf, peak_gbs, peak_kind = _peaks()
+    peak_tf, peak_tf_sust, peak_gbs, peak_kind = _peaks()
     g = torch.Generator(device=dev)
     g.manual_seed(20261202 + 7919 * rank)
 
@@ -532,9 +536,14 @@ def run_ours(args, world, rank, local):
                    "l2": "inputs larger than L2: 30-layer cache 3.45 GB + 1.7 GB activations per step",
                    "parallelism": f"replicas x{world} (independent streams)"},
         "pct_bf16_peak": value / peak_tf,
+        "pct_bf16_peak_sustained": value / peak_tf_sust,
         "latent_frames_per_s": world * F / (ms_step * 1e-3),
-        "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": attn_tf / peak_tf, "traffic": traffic, "peak_kind": f"{peak_kind} bf16 burst",
+        # the attention launches are timed inside the long timed region (seconds
+        # of steps under the power cap), so the sustained GEMM figure is the peak
+        "roofline": {"bound": "tensor", "achieved": attn_tf, "peak": peak_tf_sust, "unit": "TFLOP/s",
+                     "frac": attn_tf / peak_tf_sust, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a long step)",
+                     "frac_of_burst": attn_tf / peak_tf, "burst_peak": peak_tf,
                      "kernel": "attn_sink_window_kernel<128>", "launch_ms": attn_avg,
                      "algorithmic_flop_per_launch": ATTN_FLOP, "min_bytes_per_launch": ATTN_MIN_BYTES},
         "append": {"ms_per_layer": app_ms, "gbs": APPEND_BYTES / (app_ms * 1e-3) / 1e9,
