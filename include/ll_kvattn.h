@@ -88,7 +88,8 @@ typedef enum {
  *   capture) stay right when the graph is replayed chunk after chunk.
  *   Supported: layers, heads, tokens_per_frame, frames_per_chunk >= 1;
  *   head_dim in {64, 128}; sink_frames >= 0, window_frames >= 0,
- *   sink_frames + window_frames >= 1; (S+W)*T and F*T < 2^31; T*H*D/8 < 2^30.
+ *   sink_frames + window_frames >= 1; (S+W)*T and F*T < 2^31; T*H*D/8 and
+ *   (S+W)*T*D/8 < 2^30; heads < 32768.
  *   Returns LL_ERR_INVALID_ARG on a bad parameter or null `out`,
  *   LL_ERR_OOM if the allocation fails, LL_ERR_CUDA if no device is usable.
  *   On success *out owns the memory until ll_kv_cache_destroy.           */

@@ -269,10 +269,12 @@ __device__ __forceinline__ uint32_t bf16x2_of_f32(float lo, float hi) {
   return d;
 }
 
-template <int FMT>
+// Grid: blockIdx.y = one of the layer's 2H planes, blockIdx.x strides over the
+// plane's visible rows; VPR = D/8 vectors per row is a compile-time constant,
+// so the index arithmetic is shifts and masks in 32 bits (rows * VPR < 2^30,
+// checked at create).
+template <int FMT, int VPR>
 __global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) {
-  const int vpr = q.D >> 3;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   // visible rows as up to three slot-row ranges; rows are counted through them in order
   int r0 = 0, n0 = q.n_rows, r1 = 0, n1 = 0, r2 = 0, n2 = 0;
   if (q.ctr) {
@@ -280,23 +282,25 @@ __global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) 
     const HeldFrames hf = held_frames(__ldcg(&q.ctr->p), __ldcg(&q.ctr->shot_fill), ring_count,
                                       __ldcg(&q.ctr->ring_start), q.G, q.W);
     const FrameRanges fr = visible_ranges(hf, ring_count, q.G, q.Ss, q.W);
-    n0 = 0;
-    if (fr.n > 0) { r0 = fr.start[0] * q.T; n0 = fr.len[0] * q.T; }
-    if (fr.n > 1) { r1 = fr.start[1] * q.T; n1 = fr.len[1] * q.T; }
-    if (fr.n > 2) { r2 = fr.start[2] * q.T; n2 = fr.len[2] * q.T; }
+    r0 = fr.start[0] * q.T;
+    n0 = fr.len[0] * q.T;
+    r1 = fr.start[1] * q.T;
+    n1 = fr.len[1] * q.T;
+    r2 = fr.start[2] * q.T;
+    n2 = fr.len[2] * q.T;
   }
-  const int n_rows = n0 + n1 + n2;
-  const long long total_vec = static_cast<long long>(2 * q.H) * n_rows * vpr;
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < total_vec; i += stride) {
-    const int vec = static_cast<int>(i % vpr);
-    const long long pr = i / vpr;                       // (local plane, visible row)
-    const int vr = static_cast<int>(pr % n_rows);
-    const int lp = static_cast<int>(pr / n_rows);       // 0 .. 2H-1
+  const int total = (n0 + n1 + n2) * VPR;          // vectors of this plane
+  const int lp = blockIdx.y;                        // 0 .. 2H-1
+  const long long src_plane = static_cast<long long>(q.plane0 + lp) * q.slots;
+  const long long dst_plane = static_cast<long long>(lp) * q.slots;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
+    const int vec = i % VPR;
+    const int vr = i / VPR;                         // visible row
     const int row = vr < n0 ? r0 + vr : (vr < n0 + n1 ? r1 + (vr - n0) : r2 + (vr - n0 - n1));
-    const long long src_row = static_cast<long long>(q.plane0 + lp) * q.slots + row;
+    const long long src_row = src_plane + row;
     uint32_t o[4];
     if constexpr (FMT == FMT_FP8) {
-      const uint2 c = __ldg(reinterpret_cast<const uint2 *>(q.data + src_row * q.D) + vec);
+      const uint2 c = __ldg(reinterpret_cast<const uint2 *>(q.data + src_row * (VPR * 8)) + vec);
       const float s = __ldg(reinterpret_cast<const float *>(q.scales) + src_row);
       const uint32_t w[2] = {c.x, c.y};
 #pragma unroll
@@ -306,8 +310,8 @@ __global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) 
         o[k] = bf16x2_of_f32(f.x * s, f.y * s);
       }
     } else {
-      const uint32_t c = __ldg(reinterpret_cast<const uint32_t *>(q.data + src_row * (q.D / 2)) + vec);
-      const uint32_t sb = __ldg(q.scales + src_row * (q.D / 16) + (vec >> 1));
+      const uint32_t c = __ldg(reinterpret_cast<const uint32_t *>(q.data + src_row * (VPR * 4)) + vec);
+      const uint32_t sb = __ldg(q.scales + src_row * (VPR / 2) + (vec >> 1));
       const uint32_t s2 = f16x2_of_e4m3x2(sb * 0x101u);   // the block scale in both halves
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) 
         o[k] = bf16x2_of_f32(f.x, f.y);
       }
     }
-    q.view[(static_cast<long long>(lp) * q.slots + row) * vpr + vec] = make_uint4(o[0], o[1], o[2], o[3]);
+    q.view[(dst_plane + row) * VPR + vec] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 

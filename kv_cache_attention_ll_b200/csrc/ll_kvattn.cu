@@ -138,6 +138,25 @@ ll_status launch_attn(const llk::AttnParams &prm, int grid, cudaStream_t stream)
 
 // Quantised caches: the layer's held rows of K and V (their number follows the
 // layer's device counter), dequantised into the cache's bf16 view.
+// Grid (x, 2H): x-blocks stride over one plane's visible rows, one y per plane;
+// about 8 blocks of 256 threads per SM in all.
+ll_status launch_dequant_kernel(const llk::DequantParams &q, ll_kv_dtype dtype, int device, cudaStream_t stream) {
+  const long long plane_blocks = (static_cast<long long>(q.slots) * (q.D / 8) + 255) / 256;
+  const long long target = static_cast<long long>(num_sms(device)) * 8;
+  long long gx = (target + 2 * q.H - 1) / (2 * q.H);
+  if (gx > plane_blocks) gx = plane_blocks;
+  if (gx < 1) gx = 1;
+  const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(2 * q.H));
+  if (dtype == LL_KV_FP8_E4M3) {
+    if (q.D == 128) llk::kv_dequant_kernel<llk::FMT_FP8, 16><<<grid, 256, 0, stream>>>(q);
+    else llk::kv_dequant_kernel<llk::FMT_FP8, 8><<<grid, 256, 0, stream>>>(q);
+  } else {
+    if (q.D == 128) llk::kv_dequant_kernel<llk::FMT_NVFP4, 16><<<grid, 256, 0, stream>>>(q);
+    else llk::kv_dequant_kernel<llk::FMT_NVFP4, 8><<<grid, 256, 0, stream>>>(q);
+  }
+  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
 ll_status launch_dequant(ll_kv_cache *c, int layer, cudaStream_t stream) {
   llk::DequantParams q;
   q.data = c->data;
@@ -153,14 +172,7 @@ ll_status launch_dequant(ll_kv_cache *c, int layer, cudaStream_t stream) {
   q.W = c->W;
   q.T = c->T;
   q.plane0 = layer * 2 * c->H;
-  long long blocks = (static_cast<long long>(2 * c->H) * c->slots * (c->D / 8) + 255) / 256;
-  const long long cap = static_cast<long long>(num_sms(c->device)) * 8;
-  if (blocks > cap) blocks = cap;
-  if (c->dtype == LL_KV_FP8_E4M3)
-    llk::kv_dequant_kernel<llk::FMT_FP8><<<static_cast<int>(blocks), 256, 0, stream>>>(q);
-  else
-    llk::kv_dequant_kernel<llk::FMT_NVFP4><<<static_cast<int>(blocks), 256, 0, stream>>>(q);
-  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+  return launch_dequant_kernel(q, c->dtype, c->device, stream);
 }
 
 // Grid: one x-block per (source layer, source frame) pair, y-blocks striding
@@ -245,6 +257,7 @@ ll_status ll_kv_cache_create_multishot(int layers, int heads, int head_dim, int 
   const long long tq = static_cast<long long>(frames_per_chunk) * tokens_per_frame;
   if (slots >= (1ll << 31) || tq >= (1ll << 31)) return LL_ERR_INVALID_ARG;
   if (static_cast<long long>(tokens_per_frame) * heads * (head_dim / 8) >= (1ll << 30)) return LL_ERR_INVALID_ARG;
+  if (slots * (head_dim / 8) >= (1ll << 30) || heads >= 32768) return LL_ERR_INVALID_ARG;
   const long long planes = static_cast<long long>(layers) * 2 * heads;
   if (planes >= (1ll << 31)) return LL_ERR_INVALID_ARG;
 
@@ -591,6 +604,7 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
   const long long slots = static_cast<long long>(sink_frames + window_frames) * tokens_per_frame;
   const long long tq = static_cast<long long>(frames_per_chunk) * tokens_per_frame;
   if (slots >= (1ll << 31) || tq >= (1ll << 31)) return LL_ERR_INVALID_ARG;
+  if (slots * (head_dim / 8) >= (1ll << 30) || heads >= 32768) return LL_ERR_INVALID_ARG;
   // the view of the layer must fit the static scratch
   const unsigned long long view_bytes = 2ull * heads * static_cast<unsigned long long>(slots) * head_dim * 2;
   if (view_bytes > LL_NOALLOC_SCRATCH_BYTES) return LL_ERR_INVALID_ARG;
@@ -627,14 +641,8 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
     dq.W = window_frames;
     dq.T = tokens_per_frame;
     dq.plane0 = 0;
-    long long blocks = (static_cast<long long>(2 * heads) * n_cache * (head_dim / 8) + 255) / 256;
-    const long long cap = static_cast<long long>(num_sms(dev)) * 8;
-    if (blocks > cap) blocks = cap;
-    if (kv_dtype == LL_KV_FP8_E4M3)
-      llk::kv_dequant_kernel<llk::FMT_FP8><<<static_cast<int>(blocks), 256, 0, st>>>(dq);
-    else
-      llk::kv_dequant_kernel<llk::FMT_NVFP4><<<static_cast<int>(blocks), 256, 0, st>>>(dq);
-    if (cudaGetLastError() != cudaSuccess) return LL_ERR_CUDA;
+    const ll_status ds = launch_dequant_kernel(dq, kv_dtype, dev, st);
+    if (ds != LL_OK) return ds;
     long long tail_end = (static_cast<long long>(n_cache) + kKeyTile - 1) / kKeyTile * kKeyTile;
     if (tail_end > slots) tail_end = slots;
     if (tail_end > n_cache) {
