@@ -122,11 +122,13 @@ int num_sms(int device) {
 template <int D>
 ll_status launch_attn(const llk::AttnParams &prm, int grid, cudaStream_t stream) {
   using C = llk::AttnCfg<D>;
-  static std::atomic<unsigned> configured_mask{0};
+  // the shared-memory limit is raised once per device (devices 0..63 remembered;
+  // any other device sets it on every call)
+  static std::atomic<unsigned long long> configured_mask{0};
   int dev = 0;
-  cudaGetDevice(&dev);
-  const unsigned bit = 1u << (dev & 31);
-  if (!(configured_mask.load() & bit)) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
+  const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+  if (!bit || !(configured_mask.load() & bit)) {
     if (cudaFuncSetAttribute(llk::attn_sink_window_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM_ALLOC) != cudaSuccess)
       return LL_ERR_CUDA;

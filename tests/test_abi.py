@@ -84,3 +84,27 @@ def test_allocation_failure_hook_reports_oom_and_leaks_nothing():
     finally:
         del os.environ["LL_KVATTN_TEST_FAIL_ALLOC"]
     assert lib.ll_allocation_count() == before
+
+
+@pytest.mark.parametrize("args", [
+    (1, 2, 64, 16, 3, 3, -1, 6, 0),          # negative shot sink
+    (1, 2, 64, 16, 3, 0, 0, 0, 0),           # no frame slots at all
+    (1, 32768, 64, 16, 3, 3, 3, 6, 0),       # too many heads for the dequantise grid
+    (1, 1, 128, 1 << 25, 1, 3, 3, 2, 0),     # a plane of 2^30 or more vectors
+    (1, 2, 64, 16, 3, 3, 3, 6, 3),           # unknown dtype
+])
+def test_multishot_create_rejects_bad_arguments_before_cuda(args):
+    import kv_cache_attention_ll_b200 as ll
+    lib = ll.raw_lib()
+    h = ctypes.c_void_p(1234)
+    assert lib.ll_kv_cache_create_multishot(*args, ctypes.byref(h)) == ll.LL_ERR_INVALID_ARG
+    assert h.value is None
+
+
+def test_multishot_calls_reject_null_cache():
+    import kv_cache_attention_ll_b200 as ll
+    lib = ll.raw_lib()
+    g = ctypes.c_int()
+    assert lib.ll_kv_shot_begin(None, -1, 0, None) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_kv_cache_held(None, 0, ctypes.byref(g), None, None) == ll.LL_ERR_INVALID_ARG
+    assert lib.ll_debug_wait_selftest(None, None) == ll.LL_ERR_INVALID_ARG
