@@ -514,6 +514,33 @@ def run_ours(args, world, rank, local):
         res["speedup"] = res["full_causal"]["attn_ms_total"] / res["sink_window"]["attn_ms_total"]
         sweep["full_causal_vs_sink_window_40_chunks"] = res
 
+    # ---- fused append: the same step with one launch per layer (attention and
+    # append together) on a cache with F spare ring slots
+    fused = None
+    if not args.no_fused:
+        fc = ll.ll_kv_cache_create_fused(L, H, D, T, F, S, 0, W)
+        for c in range((S + W + F - 1) // F + 1):
+            for l in range(L):
+                ll.ll_kv_append(fc, l, ks[l], vs[l], stream)
+
+        def fstep():
+            for l in range(L):
+                ll.ll_attn_sink_window_append(qs[l], ks[l], vs[l], fc, l, outs[l], stream)
+
+        for _ in range(3):
+            fstep()
+        torch.cuda.synchronize(dev)
+        _barrier(world)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fstep()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        f_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        fused = {"ms_per_step": f_ms, "value": world * ATTN_FLOP * L / (f_ms * 1e-3) / 1e12, "launches_per_step": L,
+                 "cache_gb": ll.ll_kv_cache_info(fc, 0)[1] / 1e9, "device_status": ll.ll_debug_status(fc)}
+        fc.close()
+
     # ---- several shots (global sink + per-shot sink + window), same 12-frame
     # budget as the headline stack: global 3 + shot 3 + window 6. A shot starts
     # every 8 chunks; every second start also restarts the window, so the
@@ -588,6 +615,7 @@ def run_ours(args, world, rank, local):
         "single_layer": single,
         "long_rollout": sweep,
         "multishot": multishot,
+        "fused_append_step": fused,
         "device_status": status,
     }
     if rank == 0:
@@ -607,6 +635,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the window sweep / full-causal leg")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
     ap.add_argument("--no-multishot", action="store_true", help="skip the multi-shot cache leg")
+    ap.add_argument("--no-fused", action="store_true", help="skip the fused attention + append leg")
     ap.add_argument("--layers", type=int, default=30, help="stack depth (30 = the Wan-1.3B stack)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="CPU seconds the reference arm spends in total (bounded sample per step)")

@@ -113,6 +113,20 @@ LL_API ll_status ll_kv_cache_create_multishot(int layers, int heads, int head_di
                                               int frames_per_chunk, int global_sink_frames, int shot_sink_frames,
                                               int window_frames, ll_kv_dtype kv_dtype, ll_kv_cache **out);
 
+/* ll_kv_cache_create_fused - a cache that ll_attn_sink_window_append can use:
+ *   as ll_kv_cache_create_multishot, but the ring has F spare slots (W + F
+ *   in all), so per layer and K/V plane the layout is [H][(G+Ss+W+F)*T][D].
+ *   The window is still the last W ring frames; the spare slots hold frames
+ *   that have just left it. That is what lets one launch attend over the
+ *   window and store the chunk: the chunk's frames land in slots the launch
+ *   does not read. Costs F frames of memory per layer and K/V (25 % at chunk
+ *   3, sink 3, window 9). Every other call works on it as on any cache.
+ *   The pages describe no such layout: it exists only so that attention and
+ *   append can share one launch.                                             */
+LL_API ll_status ll_kv_cache_create_fused(int layers, int heads, int head_dim, int tokens_per_frame,
+                                          int frames_per_chunk, int global_sink_frames, int shot_sink_frames,
+                                          int window_frames, ll_kv_dtype kv_dtype, ll_kv_cache **out);
+
 /* ll_kv_shot_begin - a new shot starts with the next appended chunk.
  *   layer: 0..L-1, or -1 for all layers. Empties the shot sink (its frames are
  *   no longer attended; the next Ss non-global frames refill it). With
@@ -177,6 +191,16 @@ LL_API ll_status ll_kv_recache_write(ll_kv_cache *cache, int layer, const void *
  *   Pages: dpshk.com sec. 五/六; techwalker.com sec. 四/六; wmrh.cn sec. 6.  */
 LL_API ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cur,
                               ll_kv_cache *cache, int layer, void *out, ll_stream_t stream);
+
+/* ll_attn_sink_window_append - ll_attn_sink_window followed by ll_kv_append of
+ *   the same chunk, in one launch: the results (out, the cache bytes, the
+ *   counters) are those of the two calls in that order. Two otherwise idle
+ *   warps of each CTA store (and for FP8/NVFP4 quantise) that CTA's rows of
+ *   k_cur/v_cur. Needs a cache made by ll_kv_cache_create_fused; any other
+ *   cache returns LL_ERR_UNSUPPORTED. Arguments and errors as for
+ *   ll_attn_sink_window. Pages: as for the two calls it fuses.               */
+LL_API ll_status ll_attn_sink_window_append(const void *q, const void *k_cur, const void *v_cur,
+                                            ll_kv_cache *cache, int layer, void *out, ll_stream_t stream);
 
 /* ll_kv_cache_destroy - free all memory of the cache (NULL is a no-op).
  *   Synchronises the device first so that no enqueued work still uses it.  */

@@ -44,6 +44,8 @@ _sig = {
     "ll_kv_cache_create_multishot": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
     "ll_kv_shot_begin": (_i, [_vp, _i, _i, _vp]),
     "ll_kv_cache_held": (_i, [_vp, _i, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "ll_kv_cache_create_fused": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
+    "ll_attn_sink_window_append": (_i, [_vp, _vp, _vp, _vp, _i, _vp, _vp]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -143,6 +145,27 @@ def ll_kv_cache_create_multishot(layers: int, heads: int, head_dim: int, tokens_
                     window_frames, kv_dtype)
     cache.shot_sink_frames = shot_sink_frames
     return cache
+
+
+def ll_kv_cache_create_fused(layers: int, heads: int, head_dim: int, tokens_per_frame: int, frames_per_chunk: int,
+                             global_sink_frames: int, shot_sink_frames: int, window_frames: int,
+                             kv_dtype="bf16") -> KVCache:
+    """A cache with F spare ring slots, for ll_attn_sink_window_append."""
+    dt = _DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
+    h = _vp()
+    _check(_lib.ll_kv_cache_create_fused(layers, heads, head_dim, tokens_per_frame, frames_per_chunk,
+                                         global_sink_frames, shot_sink_frames, window_frames, dt, ctypes.byref(h)),
+           "ll_kv_cache_create_fused")
+    cache = KVCache(h.value, layers, heads, head_dim, tokens_per_frame, frames_per_chunk, global_sink_frames,
+                    window_frames, kv_dtype)
+    cache.shot_sink_frames = shot_sink_frames
+    return cache
+
+
+def ll_attn_sink_window_append(q, k_cur, v_cur, cache: KVCache, layer: int, out, stream=None):
+    """Attention of the chunk, then its append, in one launch (fused caches)."""
+    _check(_lib.ll_attn_sink_window_append(_ptr(q), _ptr(k_cur), _ptr(v_cur), cache.handle, layer, _ptr(out),
+                                           _stream(stream)), "ll_attn_sink_window_append")
 
 
 def ll_kv_shot_begin(cache: KVCache, layer: int = -1, clear_window: bool = False, stream=None):

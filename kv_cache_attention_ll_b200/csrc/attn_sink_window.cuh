@@ -23,7 +23,9 @@
 //   warps 4-7  softmax warpgroup 1
 //   warp 8     TMA producer (Q once, then K and V tiles into an NST-deep ring)
 //   warp 9     TMEM allocator and tcgen05.mma issuer
-//   warps 10-11 idle (they complete the third warpgroup for register reallocation)
+//   warps 10-11 idle (they complete the third warpgroup for register reallocation),
+//              or, when the call also appends (fused append), they store this
+//              CTA's 128 own-chunk rows of k_cur/v_cur of head h into the cache
 //
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+D),
 // O1 [256+D, 256+2D). P_g (bf16) overwrites the first 64 columns of S_g and is
@@ -37,6 +39,7 @@
 #include <cuda_bf16.h>
 
 #include "cache_layout.cuh"
+#include "kv_scatter.cuh"
 #include "sm100_ptx.cuh"
 
 namespace llk {
@@ -52,7 +55,19 @@ struct AttnParams {
   int H;
   int Tq;
   int n_cache;           // visible cache keys when ctr is null
-  int G, Ss, W, T;       // global sink, shot sink, window frames; tokens per frame (with ctr)
+  int G, Ss, W, R, T;    // global sink, shot sink, window frames, ring slots; tokens per frame (with ctr)
+  // fused append (append != 0): the chunk's own K/V also go into the cache, in
+  // the same launch; needs R >= W + F so that no written slot is one this
+  // launch reads. The last CTA to finish advances the layer's counters.
+  int append;
+  int fmt;               // cache storage format (CacheFormat)
+  int F;                 // frames per chunk
+  int plane_k_cache;     // (l*2 + 0) * H in the cache itself (plane_k may address a bf16 view)
+  int slots;             // rows per cache plane
+  const uint4 *kcur, *vcur;  // k_cur / v_cur as 16-byte vectors
+  uint8_t *cache_data, *cache_scales;
+  LayerCtr *ctr_rw;      // the layer's counters, advanced by the last CTA
+  unsigned *done;        // the layer's completion count (zero between launches)
   int plane_k;           // (l*2 + 0) * H : plane of head 0 of this layer's K
   int plane_v;           // (l*2 + 1) * H
   int num_q_tiles;
@@ -80,9 +95,10 @@ struct AttnCfg {
   // m[2][128], l[2][128] of the epilogue merge reuse the Q tile: by then every
   // MMA (all of which read Q before the last PV) has completed
   static constexpr int OFF_STATS = OFF_Q;
-  static constexpr int SMEM_BYTES = OFF_RANGES + 64;
+  static constexpr int OFF_CTR = OFF_RANGES + 64;           // counters seen at launch (fused append)
+  static constexpr int SMEM_BYTES = OFF_CTR + 32;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;      // slack for 1024-byte alignment
-  static constexpr int THREADS = 384;   // 3 warpgroups; warps 10-11 idle
+  static constexpr int THREADS = 384;   // 3 warpgroups; warps 10-11 idle unless the call appends
   // registers: launched with 384 x 168 = 64512; the producer/MMA warpgroup drops
   // to 64 and the softmax warpgroups rise to 216: 128*64 + 256*216 = 63488 <= 64512
   static constexpr uint32_t REGS_SOFTMAX = 216;
@@ -115,7 +131,7 @@ __device__ __forceinline__ KeyRanges visible_key_ranges(const AttnParams &prm) {
     const long long ring_count = __ldcg(&prm.ctr->ring_count);
     const HeldFrames hf = held_frames(__ldcg(&prm.ctr->p), __ldcg(&prm.ctr->shot_fill), ring_count,
                                       __ldcg(&prm.ctr->ring_start), prm.G, prm.W);
-    const FrameRanges fr = visible_ranges(hf, ring_count, prm.G, prm.Ss, prm.W);
+    const FrameRanges fr = visible_ranges(hf, ring_count, prm.G, prm.Ss, prm.R);
     k.r0 = fr.start[0] * prm.T;
     k.n0 = fr.len[0] * prm.T;
     k.r1 = fr.start[1] * prm.T;
@@ -178,7 +194,14 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
   volatile KeyRanges *kr = reinterpret_cast<volatile KeyRanges *>(smem + C::OFF_RANGES);
   const int nown = (prm.Tq + C::BN - 1) / C::BN;
 
+  LayerCtr *ctr_seen = reinterpret_cast<LayerCtr *>(smem + C::OFF_CTR);
   if (threadIdx.x == 0) {
+    if (prm.append) {
+      // the counters as this CTA sees them, read before its completion count
+      ctr_seen->p = __ldcg(&prm.ctr->p);
+      ctr_seen->ring_count = __ldcg(&prm.ctr->ring_count);
+      ctr_seen->shot_fill = __ldcg(&prm.ctr->shot_fill);
+    }
     const KeyRanges k = visible_key_ranges(prm);
     kr->r0 = k.r0; kr->n0 = k.n0; kr->r1 = k.r1; kr->n1 = k.n1; kr->r2 = k.r2; kr->n2 = k.n2;
     kr->t1 = k.t1; kr->t2 = k.t2; kr->nc = k.nc;
@@ -274,6 +297,43 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
         mbar_wait_drain(v_full + j % C::NST, (j / C::NST) & 1);
     }
     __syncwarp();
+  } else if (warp >= 10) {
+    if (prm.append) {
+      // ---------------------------------------------------- fused append
+      // Own-chunk rows q0 .. q0+127 of head h: each (token, head) row is D/8
+      // consecutive lanes; the trip count is uniform, so the quantising
+      // formats' row shuffles always see whole warps.
+      constexpr int VPR = D / 8;
+      const int tid = threadIdx.x - 320;                       // 0 .. 63
+      const int rows = min(C::BM, prm.Tq - q0);
+      const long long p = ctr_seen->p, ring_count = ctr_seen->ring_count;
+      const int shot_fill = ctr_seen->shot_fill;
+      const long long plane_k = prm.plane_k_cache + h, plane_v = plane_k + prm.H;
+      for (int base = 0; base < C::BM * VPR; base += 64) {
+        const int i = base + tid;
+        const int r = i / VPR, vec = i % VPR;
+        const int t = q0 + r;                                  // token of the chunk
+        const int fi = t / prm.T;
+        const int slot = r < rows ? append_slot(p, shot_fill, ring_count, prm.G, prm.Ss, prm.R, prm.F, fi) : -1;
+        const bool act = slot >= 0;
+        const long long drow = static_cast<long long>(slot) * prm.T + (t - fi * prm.T);
+        uint4 vk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+        if (act) {
+          const long long src = (static_cast<long long>(t) * prm.H + h) * VPR + vec;
+          vk = __ldg(prm.kcur + src);
+          vv = __ldg(prm.vcur + src);
+        }
+        if (prm.fmt == FMT_FP8)
+          store_kv_vec<FMT_FP8>(prm.cache_data, prm.cache_scales, plane_k, plane_v, prm.slots, drow, D, vec, vk, vv,
+                                act);
+        else if (prm.fmt == FMT_NVFP4)
+          store_kv_vec<FMT_NVFP4>(prm.cache_data, prm.cache_scales, plane_k, plane_v, prm.slots, drow, D, vec, vk, vv,
+                                  act);
+        else
+          store_kv_vec<FMT_BF16>(prm.cache_data, prm.cache_scales, plane_k, plane_v, prm.slots, drow, D, vec, vk, vv,
+                                 act);
+      }
+    }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop converged (operands stay warp-uniform);
@@ -481,6 +541,22 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (prm.append && threadIdx.x == 0) {
+    // the last CTA to finish advances the layer's counters; every CTA read them
+    // at its start, before its increment of the completion count
+    __threadfence();
+    const unsigned prev = atomicAdd(prm.done, 1u);
+    if (prev == gridDim.x - 1) {
+      int fill;
+      long long rc;
+      append_advance(ctr_seen->p, ctr_seen->shot_fill, ctr_seen->ring_count, prm.G, prm.Ss, prm.F, &fill, &rc);
+      prm.ctr_rw->p = ctr_seen->p + prm.F;
+      prm.ctr_rw->shot_fill = fill;
+      prm.ctr_rw->ring_count = rc;
+      *prm.done = 0;
+      __threadfence();
+    }
   }
 #undef TM_S
 #undef TM_O

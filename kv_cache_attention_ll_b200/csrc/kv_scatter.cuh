@@ -43,7 +43,7 @@ struct ScatterParams {
   int layer0;                // first destination layer
   int n_frames;              // frames per source layer
   int mode;                  // ScatterMode
-  int G, Ss, W, F;           // cache geometry: global sink, shot sink, window, chunk frames
+  int G, Ss, W, R, F;        // cache geometry: global sink, shot sink, window, ring slots, chunk frames
   int first;                 // recache: first logical frame
   LayerCtr *ctr;             // per-layer counters (device); append advances its layer's
   unsigned *done;            // per-layer count of finished append blocks (zero between launches),
@@ -94,6 +94,74 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&x)[8]) {
   }
 }
 
+// Stores one 16-byte vector (8 values) of K and the same vector of V of one
+// (token, head) row at row `drow` of planes plane_k / plane_v, quantising for
+// FP8 (per-row scale) and NVFP4 (16-value blocks). The D/8 lanes of a row must
+// be consecutive lanes of the warp, and every lane of the warp must call it:
+// the quantising formats reduce with shuffles. Lanes with act = false take
+// part in the shuffles and store nothing.
+template <int FMT>
+__device__ __forceinline__ void store_kv_vec(uint8_t *data, uint8_t *scales, long long plane_k, long long plane_v,
+                                             int slots, long long drow, int D, int vec, uint4 vk, uint4 vv,
+                                             bool act) {
+  const int vpr = D >> 3;
+  if constexpr (FMT == FMT_BF16) {
+    if (act) {
+      uint4 *dk = reinterpret_cast<uint4 *>(data) + (plane_k * slots + drow) * vpr + vec;
+      uint4 *dv = reinterpret_cast<uint4 *>(data) + (plane_v * slots + drow) * vpr + vec;
+      *dk = vk;
+      *dv = vv;
+    }
+  } else if constexpr (FMT == FMT_FP8) {
+    // per (token, head) row: scale = amax/448 (1 if amax == 0), codes = E4M3(x * (1/scale))
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+      float x[8];
+      bf16x8_to_f32(kv == 0 ? vk : vv, x);
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+      for (int o = 1; o < vpr; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float scale = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+      const float inv = __fdiv_rn(1.0f, scale);
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(x[e], inv);
+      const uint2 codes = e4m3x8(y);
+      if (act) {
+        const long long plane = kv == 0 ? plane_k : plane_v;
+        uint2 *dc = reinterpret_cast<uint2 *>(data + (plane * slots + drow) * D) + vec;
+        *dc = codes;
+        if (vec == 0) reinterpret_cast<float *>(scales)[plane * slots + drow] = scale;
+      }
+    }
+  } else {
+    // NVFP4: per 16-value block (two lanes): sb = E4M3(amax/6); codes = E2M1(x / sb), 0 if sb == 0
+#pragma unroll
+    for (int kv = 0; kv < 2; ++kv) {
+      float x[8];
+      bf16x8_to_f32(kv == 0 ? vk : vv, x);
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      float sv[8] = {__fdiv_rn(amax, 6.0f), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const uint32_t sb_code = e4m3x8(sv).x & 0xFFu;
+      const float sb = e4m3_to_f32(sb_code);
+      float y[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] = sb == 0.f ? 0.f : __fdiv_rn(x[e], sb);
+      const uint32_t codes = sb == 0.f ? 0u : e2m1x8(y);
+      if (act) {
+        const long long plane = kv == 0 ? plane_k : plane_v;
+        uint32_t *dc = reinterpret_cast<uint32_t *>(data + (plane * slots + drow) * (D / 2)) + vec;
+        *dc = codes;
+        if ((vec & 1) == 0) scales[(plane * slots + drow) * (D / 16) + (vec >> 1)] = static_cast<uint8_t>(sb_code);
+      }
+    }
+  }
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) {
   const int vpr = q.D >> 3;                    // vectors per (token, head) row: 8 or 16
@@ -119,13 +187,13 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
   const int shot_fill = blk_ctr.shot_fill;
   int slot;
   if (q.mode == SCATTER_APPEND) {
-    slot = append_slot(p, shot_fill, ring_count, q.G, q.Ss, q.W, q.F, fi);
+    slot = append_slot(p, shot_fill, ring_count, q.G, q.Ss, q.R, q.F, fi);
   } else {
     const HeldFrames hf = held_frames(p, shot_fill, ring_count, ring_start, q.G, q.W);
     // recache of frames the layer does not hold: nothing of that layer is written
     const bool reject = q.first + q.n_frames > hf.g + hf.sf + hf.w;
     if (reject && fi == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(q.err, KID_SCATTER | ERR_RANGE);
-    slot = reject ? -1 : logical_slot(hf, ring_count, q.G, q.Ss, q.W, q.first + fi);
+    slot = reject ? -1 : logical_slot(hf, ring_count, q.G, q.Ss, q.R, q.first + fi);
   }
   const long long src0 = static_cast<long long>(blockIdx.x) * q.frame_vec;   // first vector of the frame
   const int stride = gridDim.y * blockDim.x;
@@ -147,61 +215,7 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
       vk = __ldg(q.src_k + src0 + ic);
       vv = __ldg(q.src_v + src0 + ic);
     }
-    if constexpr (FMT == FMT_BF16) {
-      if (act) {
-        uint4 *dk = reinterpret_cast<uint4 *>(q.data) + (plane_k * q.slots + drow) * vpr + vec;
-        uint4 *dv = reinterpret_cast<uint4 *>(q.data) + (plane_v * q.slots + drow) * vpr + vec;
-        *dk = vk;
-        *dv = vv;
-      }
-    } else if constexpr (FMT == FMT_FP8) {
-      // per (token, head) row: scale = amax/448 (1 if amax == 0), codes = E4M3(x * (1/scale))
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-        float x[8];
-        bf16x8_to_f32(kv == 0 ? vk : vv, x);
-        float amax = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
-        for (int o = 1; o < vpr; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        const float scale = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
-        const float inv = __fdiv_rn(1.0f, scale);
-        float y[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(x[e], inv);
-        const uint2 codes = e4m3x8(y);
-        if (act) {
-          const long long plane = kv == 0 ? plane_k : plane_v;
-          uint2 *dc = reinterpret_cast<uint2 *>(q.data + (plane * q.slots + drow) * q.D) + vec;
-          *dc = codes;
-          if (vec == 0) reinterpret_cast<float *>(q.scales)[plane * q.slots + drow] = scale;
-        }
-      }
-    } else {
-      // NVFP4: per 16-value block (two lanes): sb = E4M3(amax/6); codes = E2M1(x / sb), 0 if sb == 0
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-        float x[8];
-        bf16x8_to_f32(kv == 0 ? vk : vv, x);
-        float amax = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
-        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-        float sv[8] = {__fdiv_rn(amax, 6.0f), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const uint32_t sb_code = e4m3x8(sv).x & 0xFFu;
-        const float sb = e4m3_to_f32(sb_code);
-        float y[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] = sb == 0.f ? 0.f : __fdiv_rn(x[e], sb);
-        const uint32_t codes = sb == 0.f ? 0u : e2m1x8(y);
-        if (act) {
-          const long long plane = kv == 0 ? plane_k : plane_v;
-          uint32_t *dc = reinterpret_cast<uint32_t *>(q.data + (plane * q.slots + drow) * (q.D / 2)) + vec;
-          *dc = codes;
-          if ((vec & 1) == 0) q.scales[(plane * q.slots + drow) * (q.D / 16) + (vec >> 1)] = static_cast<uint8_t>(sb_code);
-        }
-      }
-    }
+    store_kv_vec<FMT>(q.data, q.scales, plane_k, plane_v, q.slots, drow, q.D, vec, vk, vv, act);
   }
   if (q.mode == SCATTER_APPEND) {
     // the last block to finish advances the counters; every block read them
@@ -249,7 +263,7 @@ struct DequantParams {
   uint4 *view;             // [2H][slots][D] bf16
   const LayerCtr *ctr;     // the layer's counters, or null: then rows [0, n_rows) are converted
   int H, D, slots, n_rows;
-  int G, Ss, W, T;         // with ctr: the visible frame ranges of cache_layout.cuh are converted
+  int G, Ss, W, R, T;      // with ctr: the visible frame ranges of cache_layout.cuh are converted
   int plane0;              // first plane of the layer: layer * 2H
 };
 
@@ -281,7 +295,7 @@ __global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) 
     const long long ring_count = __ldcg(&q.ctr->ring_count);
     const HeldFrames hf = held_frames(__ldcg(&q.ctr->p), __ldcg(&q.ctr->shot_fill), ring_count,
                                       __ldcg(&q.ctr->ring_start), q.G, q.W);
-    const FrameRanges fr = visible_ranges(hf, ring_count, q.G, q.Ss, q.W);
+    const FrameRanges fr = visible_ranges(hf, ring_count, q.G, q.Ss, q.R);
     r0 = fr.start[0] * q.T;
     n0 = fr.len[0] * q.T;
     r1 = fr.start[1] * q.T;

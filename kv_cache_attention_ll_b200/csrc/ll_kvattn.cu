@@ -28,9 +28,10 @@
 struct ll_kv_cache {
   int L, H, D, T, F, S, W;
   int Ss;                     // shot-sink frames (0: a single-shot cache)
+  int R;                      // ring slots: W, or W + F for a cache made for fused append
   ll_kv_dtype dtype;
   int device;
-  long long slots;            // (S+Ss+W)*T rows per plane
+  long long slots;            // (S+Ss+R)*T rows per plane
   uint8_t *base;              // the one allocation
   size_t bytes;               // its size
   uint8_t *data;              // [L][2][H][slots][row bytes]
@@ -100,6 +101,19 @@ bool make_act_map(CUtensorMap *m, const void *p, int Tq, int H, int D) {
 llk::HeldFrames held(const ll_kv_cache *c, int layer) {
   const llk::LayerCtr &h = c->hc[layer];
   return llk::held_frames(h.p, h.shot_fill, h.ring_count, h.ring_start, c->S, c->W);
+}
+
+// counter updates of one append of layer `layer` on the host mirror; an append
+// enqueued inside a stream capture ends the mirror's exactness
+void mirror_append(ll_kv_cache *c, int layer, cudaStreamCaptureStatus cs) {
+  llk::LayerCtr &h = c->hc[layer];
+  int fill = 0;
+  long long rc = 0;
+  llk::append_advance(h.p, h.shot_fill, h.ring_count, c->S, c->Ss, c->F, &fill, &rc);
+  h.p += c->F;
+  h.shot_fill = fill;
+  h.ring_count = rc;
+  if (cs != cudaStreamCaptureStatusNone) c->host_counters = false;
 }
 
 // the device counters of one layer (after a device-wide synchronisation)
@@ -172,6 +186,7 @@ ll_status launch_dequant(ll_kv_cache *c, int layer, cudaStream_t stream) {
   q.G = c->S;
   q.Ss = c->Ss;
   q.W = c->W;
+  q.R = c->R;
   q.T = c->T;
   q.plane0 = layer * 2 * c->H;
   return launch_dequant_kernel(q, c->dtype, c->device, stream);
@@ -212,12 +227,21 @@ llk::ScatterParams scatter_base(const ll_kv_cache *c, const void *k, const void 
   q.G = c->S;
   q.Ss = c->Ss;
   q.W = c->W;
+  q.R = c->R;
   q.F = c->F;
   q.ctr = c->ctr;
   q.done = c->done;
   q.err = c->err;
   return q;
 }
+
+ll_status attention(const void *q, const void *k_cur, const void *v_cur, ll_kv_cache *c, int layer, void *out,
+                    ll_stream_t stream, bool append);
+
+// one cache; spare_slots adds F ring slots (the layout the fused append needs)
+ll_status create_cache(int layers, int heads, int head_dim, int tokens_per_frame, int frames_per_chunk,
+                       int global_sink_frames, int shot_sink_frames, int window_frames, bool spare_slots,
+                       ll_kv_dtype kv_dtype, ll_kv_cache **out);
 
 }  // namespace
 
@@ -246,6 +270,23 @@ ll_status ll_kv_cache_create(int layers, int heads, int head_dim, int tokens_per
 ll_status ll_kv_cache_create_multishot(int layers, int heads, int head_dim, int tokens_per_frame,
                                        int frames_per_chunk, int global_sink_frames, int shot_sink_frames,
                                        int window_frames, ll_kv_dtype kv_dtype, ll_kv_cache **out) {
+  return create_cache(layers, heads, head_dim, tokens_per_frame, frames_per_chunk, global_sink_frames,
+                      shot_sink_frames, window_frames, false, kv_dtype, out);
+}
+
+ll_status ll_kv_cache_create_fused(int layers, int heads, int head_dim, int tokens_per_frame, int frames_per_chunk,
+                                   int global_sink_frames, int shot_sink_frames, int window_frames,
+                                   ll_kv_dtype kv_dtype, ll_kv_cache **out) {
+  return create_cache(layers, heads, head_dim, tokens_per_frame, frames_per_chunk, global_sink_frames,
+                      shot_sink_frames, window_frames, true, kv_dtype, out);
+}
+
+}  // extern "C"
+
+namespace {
+ll_status create_cache(int layers, int heads, int head_dim, int tokens_per_frame, int frames_per_chunk,
+                       int global_sink_frames, int shot_sink_frames, int window_frames, bool spare_slots,
+                       ll_kv_dtype kv_dtype, ll_kv_cache **out) {
   if (!out) return LL_ERR_INVALID_ARG;
   *out = nullptr;
   const int sink_frames = global_sink_frames;
@@ -254,8 +295,8 @@ ll_status ll_kv_cache_create_multishot(int layers, int heads, int head_dim, int 
   if (sink_frames < 0 || shot_sink_frames < 0 || window_frames < 0) return LL_ERR_INVALID_ARG;
   if (static_cast<long long>(sink_frames) + shot_sink_frames + window_frames < 1) return LL_ERR_INVALID_ARG;
   if (kv_dtype != LL_KV_BF16 && kv_dtype != LL_KV_FP8_E4M3 && kv_dtype != LL_KV_NVFP4) return LL_ERR_INVALID_ARG;
-  const long long slots =
-      (static_cast<long long>(sink_frames) + shot_sink_frames + window_frames) * tokens_per_frame;
+  const long long ring_slots = static_cast<long long>(window_frames) + (spare_slots ? frames_per_chunk : 0);
+  const long long slots = (static_cast<long long>(sink_frames) + shot_sink_frames + ring_slots) * tokens_per_frame;
   const long long tq = static_cast<long long>(frames_per_chunk) * tokens_per_frame;
   if (slots >= (1ll << 31) || tq >= (1ll << 31)) return LL_ERR_INVALID_ARG;
   if (static_cast<long long>(tokens_per_frame) * heads * (head_dim / 8) >= (1ll << 30)) return LL_ERR_INVALID_ARG;
@@ -293,6 +334,7 @@ ll_status ll_kv_cache_create_multishot(int layers, int heads, int head_dim, int 
   c->L = layers; c->H = heads; c->D = head_dim; c->T = tokens_per_frame; c->F = frames_per_chunk;
   c->S = sink_frames; c->W = window_frames; c->dtype = kv_dtype; c->device = dev; c->slots = slots;
   c->Ss = shot_sink_frames;
+  c->R = static_cast<int>(ring_slots);
   c->hc.assign(layers, llk::LayerCtr{0, 0, 0, 0, 0});
   c->host_counters = true;
   c->data_plane_bytes = data_plane;
@@ -337,6 +379,9 @@ ll_status ll_kv_cache_create_multishot(int layers, int heads, int head_dim, int 
   *out = c;
   return LL_OK;
 }
+}  // namespace
+
+extern "C" {
 
 ll_status ll_kv_cache_destroy(ll_kv_cache *c) {
   if (!c) return LL_OK;
@@ -414,16 +459,7 @@ ll_status ll_kv_append(ll_kv_cache *c, int layer, const void *k_cur, const void 
   q.layer0 = layer;
   q.n_frames = c->F;
   const ll_status r = launch_scatter(c, q, 1, st);
-  if (r == LL_OK) {
-    llk::LayerCtr &h = c->hc[layer];
-    int fill = 0;
-    long long rc = 0;
-    llk::append_advance(h.p, h.shot_fill, h.ring_count, c->S, c->Ss, c->F, &fill, &rc);
-    h.p += c->F;
-    h.shot_fill = fill;
-    h.ring_count = rc;
-    if (cs != cudaStreamCaptureStatusNone) c->host_counters = false;
-  }
+  if (r == LL_OK) mirror_append(c, layer, cs);
   return r;
 }
 
@@ -455,9 +491,32 @@ ll_status ll_kv_recache_write(ll_kv_cache *c, int layer, const void *k_new, cons
 
 ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cur, ll_kv_cache *c, int layer,
                               void *out, ll_stream_t stream) {
+  return attention(q, k_cur, v_cur, c, layer, out, stream, false);
+}
+
+ll_status ll_attn_sink_window_append(const void *q, const void *k_cur, const void *v_cur, ll_kv_cache *c, int layer,
+                                     void *out, ll_stream_t stream) {
+  return attention(q, k_cur, v_cur, c, layer, out, stream, true);
+}
+
+}  // extern "C"
+
+namespace {
+// attention of one layer's chunk; with append, the same launch also stores the
+// chunk in the cache (which must have F spare ring slots) and advances the
+// layer's counters, exactly as ll_kv_append after the attention would
+ll_status attention(const void *q, const void *k_cur, const void *v_cur, ll_kv_cache *c, int layer, void *out,
+                    ll_stream_t stream, bool append) {
   if (!c || layer < 0 || layer >= c->L || !q || !k_cur || !v_cur || !out) return LL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out)) return LL_ERR_INVALID_ARG;
   if (out == q || out == k_cur || out == v_cur) return LL_ERR_INVALID_ARG;
+  if (append && c->R < c->W + c->F) return LL_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (append && cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+    cudaGetLastError();
+    return LL_ERR_CUDA;
+  }
   const int Tq = c->F * c->T;
   llk::AttnParams prm;
   std::memset(&prm, 0, sizeof(prm));
@@ -474,6 +533,7 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   prm.G = c->S;
   prm.Ss = c->Ss;
   prm.W = c->W;
+  prm.R = c->R;
   prm.T = c->T;
   prm.H = c->H;
   prm.Tq = Tq;
@@ -481,14 +541,31 @@ ll_status ll_attn_sink_window(const void *q, const void *k_cur, const void *v_cu
   prm.plane_v = quantised ? c->H : (layer * 2 + 1) * c->H;
   prm.num_q_tiles = (Tq + 127) / 128;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->D)));
+  if (append) {
+    prm.append = 1;
+    prm.fmt = c->dtype == LL_KV_BF16 ? llk::FMT_BF16 : (c->dtype == LL_KV_FP8_E4M3 ? llk::FMT_FP8 : llk::FMT_NVFP4);
+    prm.F = c->F;
+    prm.plane_k_cache = layer * 2 * c->H;
+    prm.slots = static_cast<int>(c->slots);
+    prm.kcur = static_cast<const uint4 *>(k_cur);
+    prm.vcur = static_cast<const uint4 *>(v_cur);
+    prm.cache_data = c->data;
+    prm.cache_scales = c->scales;
+    prm.ctr_rw = c->ctr + layer;
+    prm.done = c->done + layer;
+  }
   const int grid = prm.num_q_tiles * c->H;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (quantised) {
     const ll_status ds = launch_dequant(c, layer, st);
     if (ds != LL_OK) return ds;
   }
-  return c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
+  const ll_status r = c->D == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
+  if (r == LL_OK && append) mirror_append(c, layer, cs);
+  return r;
 }
+}  // namespace
+
+extern "C" {
 
 // ---------------------------------------------------------------------------
 // Shot start (several shots per video): empties the shot sink of the addressed
@@ -641,6 +718,7 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
     dq.G = sink_frames;
     dq.Ss = 0;
     dq.W = window_frames;
+    dq.R = window_frames;
     dq.T = tokens_per_frame;
     dq.plane0 = 0;
     const ll_status ds = launch_dequant_kernel(dq, kv_dtype, dev, st);

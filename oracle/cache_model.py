@@ -40,6 +40,12 @@ order: global sink, shot sink (fill order), window (oldest to newest, at most
 the last W ring frames since the last window restart). With Ss = 0 and no
 shot_begin this is exactly the single-shot rule above.
 
+Spare ring slots (ring_slots = R > W): the ring has R slots and ring frame
+number i lives in slot S + Ss + (i mod R); the window is still its last W
+frames. With R = W + F the F frames a chunk appends land in slots the window
+no longer covers, so attention and append can share one launch. The held
+frames are the same as with R = W; only the slots differ.
+
 Stored formats: "bf16" raw bits; "fp8" E4M3 codes + one fp32 scale per
 (token, head) row; "nvfp4" packed E2M1 codes + one E4M3 scale per 16 values.
 Export of a layer = data of K, data of V, then (quantised formats) scales of K,
@@ -55,13 +61,15 @@ from . import quant
 class CacheModel:
     def __init__(self, layers: int, heads: int, head_dim: int, tokens_per_frame: int,
                  frames_per_chunk: int, sink_frames: int, window_frames: int, kv_dtype: str = "bf16",
-                 shot_sink_frames: int = 0):
+                 shot_sink_frames: int = 0, ring_slots: int | None = None):
         assert kv_dtype in ("bf16", "fp8", "nvfp4")
         self.L, self.H, self.D = layers, heads, head_dim
         self.T, self.F, self.S, self.W = tokens_per_frame, frames_per_chunk, sink_frames, window_frames
         self.Ss = shot_sink_frames
+        self.R = self.W if ring_slots is None else ring_slots
+        assert self.R >= self.W
         self.kv_dtype = kv_dtype
-        self.slots = (self.S + self.Ss + self.W) * self.T
+        self.slots = (self.S + self.Ss + self.R) * self.T
         shape = (layers, 2, heads, self.slots)
         if kv_dtype == "bf16":
             self.data = np.zeros(shape + (head_dim,), dtype=np.uint16)
@@ -90,9 +98,9 @@ class CacheModel:
             return slot
         idx = self.ring_count[layer]
         self.ring_count[layer] += 1
-        if self.W == 0:
+        if self.R == 0:
             return None
-        return self.S + self.Ss + idx % self.W
+        return self.S + self.Ss + idx % self.R
 
     def held(self, layer: int):
         """(global sink frames, window frames) held; see held3 for the shot sink."""
@@ -117,7 +125,7 @@ class CacheModel:
         if k < g + sf:
             return self.S + (k - g)
         idx = self.ring_count[layer] - w + (k - g - sf)
-        return self.S + self.Ss + idx % self.W
+        return self.S + self.Ss + idx % self.R
 
     # -- writes -------------------------------------------------------------
     def _store_frame(self, layer: int, kv: int, slot: int, src_bits: np.ndarray):

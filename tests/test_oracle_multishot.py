@@ -171,3 +171,30 @@ def test_attention_over_explicit_visible_frames_brute_force():
             z = sum(e)
             want = [sum(e[t] * vf[keys[t], h, d] for t in range(len(keys))) / z for d in range(D)]
             np.testing.assert_allclose(got[i, h], want, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("G,Ss,W,F,T", GEOMS)
+def test_spare_ring_slots_hold_the_same_frames(G, Ss, W, F, T):
+    """A cache whose ring has F spare slots (R = W + F, the layout that lets
+    attention and append share one launch) holds exactly the frames of the
+    plain layout, with the same bits in logical order; only slots differ. And
+    the frames a chunk appends never land in a slot the window covered just
+    before that append."""
+    H, D, n = 1, 8, 15
+    seed = mix_seed(G, Ss, W, F, 91)
+    shots = dict(_schedule(seed, n))
+    plain = CacheModel(1, H, D, T, F, G, W, shot_sink_frames=Ss)
+    spare = CacheModel(1, H, D, T, F, G, W, shot_sink_frames=Ss, ring_slots=W + F)
+    for c in range(n):
+        for m in (plain, spare):
+            if c in shots:
+                m.shot_begin(0, shots[c])
+        visible_slots = {spare.logical_slot(0, k) for k in range(spare.n_held(0))}
+        before = dict(spare.slot_frame[0])
+        k, v = _chunk(seed, c, F, T, H, D)
+        plain.append(0, k, v)
+        spare.append(0, k, v)
+        written = {sl for sl, f in spare.slot_frame[0].items() if before.get(sl) != f}
+        assert not (written & visible_slots), f"chunk {c} wrote a visible slot"
+        assert list(plain.held_frames(0, 0)) == list(spare.held_frames(0, 0))
+        np.testing.assert_array_equal(plain.logical_view(0, 0), spare.logical_view(0, 0))
