@@ -47,8 +47,8 @@ ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out
 # ncu DRAM traffic of one attention launch at this shape and the kernel sources it
 # was taken with (profiles/attn_sink_window_wan1.3b.md); reported only while the
 # kernel is unchanged.
-ATTN_TRAFFIC = 167.0e6         # mean of the two captured launches (166.6 MB, 167.4 MB)
-ATTN_TRAFFIC_SRC_SHA = "2cc1e069977cef9a"
+ATTN_TRAFFIC = 167.0e6         # mean of the two captured launches (166.95 MB, 167.0 MB)
+ATTN_TRAFFIC_SRC_SHA = "fb4e17ca4f14cda4"
 
 
 def _peaks():
@@ -66,7 +66,7 @@ def _peaks():
 
 def _kernel_sha() -> str:
     h = hashlib.sha256()
-    for f in ("attn_sink_window.cuh", "sm100_ptx.cuh", "cache_layout.cuh"):
+    for f in ("attn_sink_window.cuh", "sm100_ptx.cuh", "cache_layout.cuh", "kv_scatter.cuh"):
         with open(os.path.join(ROOT, "kv_cache_attention_ll_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
