@@ -30,6 +30,10 @@
  *   the host. Calls touching the same layer must be ordered by the caller, on
  *   one stream or with events. The host-side frame counter of a layer advances
  *   when ll_kv_append is called (enqueue order = logical order).
+ *   A cache lives on the device that was current at create: calls that launch
+ *   work on it must be made with that device current (else
+ *   LL_ERR_INVALID_ARG), and their tensors must live on that device. Calls on
+ *   one cache from several host threads must be serialised by the caller.
  *   Errors are returned, never raised or aborted; on an error nothing was
  *   enqueued unless the status is LL_ERR_CUDA (a launch failed), and the cache
  *   handle stays valid.

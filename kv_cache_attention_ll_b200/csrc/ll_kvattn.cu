@@ -72,6 +72,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Kernels of a cache run on the device that owns it: a launch on another
+// current device would reach memory of a device it may not be able to access.
+bool on_cache_device(const ll_kv_cache *c) {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev == c->device;
+}
+
 // 3-D bf16 tensor map: dims (d0 innermost, d1, d2), strides of d1 and d2 in bytes,
 // box (b0, b1, b2), 128-byte swizzle, zero fill outside the tensor.
 bool make_map_3d(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
@@ -448,6 +455,7 @@ ll_status ll_debug_status(ll_kv_cache *c, unsigned int *word, int clear, ll_stre
 ll_status ll_kv_append(ll_kv_cache *c, int layer, const void *k_cur, const void *v_cur, ll_stream_t stream) {
   if (!c || layer < 0 || layer >= c->L || !k_cur || !v_cur || !aligned16(k_cur) || !aligned16(v_cur))
     return LL_ERR_INVALID_ARG;
+  if (!on_cache_device(c)) return LL_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
@@ -467,6 +475,7 @@ ll_status ll_kv_recache_write(ll_kv_cache *c, int layer, const void *k_new, cons
                               int num_frames, ll_stream_t stream) {
   if (!c || layer < -1 || layer >= c->L || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))
     return LL_ERR_INVALID_ARG;
+  if (!on_cache_device(c)) return LL_ERR_INVALID_ARG;
   if (first_frame < 0 || num_frames < 1) return LL_ERR_INVALID_ARG;
   const int l0 = layer < 0 ? 0 : layer;
   const int nl = layer < 0 ? c->L : 1;
@@ -510,6 +519,7 @@ ll_status attention(const void *q, const void *k_cur, const void *v_cur, ll_kv_c
   if (!c || layer < 0 || layer >= c->L || !q || !k_cur || !v_cur || !out) return LL_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(out)) return LL_ERR_INVALID_ARG;
   if (out == q || out == k_cur || out == v_cur) return LL_ERR_INVALID_ARG;
+  if (!on_cache_device(c)) return LL_ERR_INVALID_ARG;
   if (append && c->R < c->W + c->F) return LL_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
@@ -583,6 +593,7 @@ __global__ void shot_begin_kernel(LayerCtr *ctr, int l0, int nl, int clear_windo
 
 extern "C" ll_status ll_kv_shot_begin(ll_kv_cache *c, int layer, int clear_window, ll_stream_t stream) {
   if (!c || layer < -1 || layer >= c->L) return LL_ERR_INVALID_ARG;
+  if (!on_cache_device(c)) return LL_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
@@ -632,7 +643,7 @@ __global__ void wait_selftest_kernel(unsigned *err) {
 }  // namespace llk
 
 extern "C" ll_status ll_debug_wait_selftest(ll_kv_cache *c, ll_stream_t stream) {
-  if (!c) return LL_ERR_INVALID_ARG;
+  if (!c || !on_cache_device(c)) return LL_ERR_INVALID_ARG;
   llk::wait_selftest_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c->err);
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
