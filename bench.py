@@ -513,6 +513,27 @@ def run_ours(args, world, rank, local):
             sc.close()
         res["speedup"] = res["full_causal"]["attn_ms_total"] / res["sink_window"]["attn_ms_total"]
         sweep["full_causal_vs_sink_window_40_chunks"] = res
+        # 320 chunks (960 latent frames) from an empty cache, sink 3 + window 9:
+        # per-chunk attention time, and the footprint checked constant (no
+        # allocation by the library, no change of free device memory)
+        sc = ll.ll_kv_cache_create(1, H, D, T, F, S, W)
+        torch.cuda.synchronize(dev)
+        n_alloc0, free0 = ll.ll_allocation_count(), torch.cuda.mem_get_info(dev)[0]
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(320)]
+        for c in range(320):
+            evs[c][0].record(stream)
+            ll.ll_attn_sink_window(q1, k1, v1, sc, 0, o1, stream)
+            evs[c][1].record(stream)
+            ll.ll_kv_append(sc, 0, k1, v1, stream)
+        torch.cuda.synchronize(dev)
+        ms = [a.elapsed_time(b) for a, b in evs]
+        sweep["rollout_320_chunks"] = {
+            "frames": 320 * F, "attn_ms_total": sum(ms),
+            "attn_ms_median_chunks_4_319": statistics.median(ms[4:]),
+            "allocation_count_constant": ll.ll_allocation_count() == n_alloc0,
+            "free_device_bytes_constant": torch.cuda.mem_get_info(dev)[0] == free0,
+            "frames_seen": ll.ll_kv_cache_info(sc, 0)[0], "cache_gb": ll.ll_kv_cache_info(sc, 0)[1] / 1e9}
+        sc.close()
 
     # ---- fused append: the same step with one launch per layer (attention and
     # append together) on a cache with F spare ring slots
