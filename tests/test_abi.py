@@ -108,3 +108,36 @@ def test_multishot_calls_reject_null_cache():
     assert lib.ll_kv_shot_begin(None, -1, 0, None) == ll.LL_ERR_INVALID_ARG
     assert lib.ll_kv_cache_held(None, 0, ctypes.byref(g), None, None) == ll.LL_ERR_INVALID_ARG
     assert lib.ll_debug_wait_selftest(None, None) == ll.LL_ERR_INVALID_ARG
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """The boundary is a C ABI: a C99 program that includes the header, takes
+    the address of every entry point and calls the ones that need no device
+    links against the library and runs."""
+    import shutil
+    import subprocess
+    import kv_cache_attention_ll_b200 as ll
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    names = _declared()
+    src = tmp_path / "use_abi.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"ll_kvattn.h\"\n"
+        "int main(void) {\n"
+        "  const void *fns[] = {" + ", ".join(f"(const void *)&{n}" for n in names) + "};\n"
+        "  ll_kv_cache *c = (ll_kv_cache *)0;\n"
+        "  if (ll_kv_cache_create(0, 1, 64, 1, 1, 1, 1, LL_KV_BF16, &c) != LL_ERR_INVALID_ARG || c) return 1;\n"
+        "  if (ll_kv_cache_destroy((ll_kv_cache *)0) != LL_OK) return 2;\n"
+        "  if (ll_allocation_count() != 0) return 3;\n"
+        "  printf(\"%s %d\\n\", ll_status_string(LL_ERR_TIMEOUT), (int)(sizeof(fns) / sizeof(fns[0])));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "use_abi"
+    libdir = os.path.dirname(ll.LIB_PATH)
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+           "-L", libdir, "-lll_kvattn", "-Wl,-rpath," + libdir]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.split() == ["in-kernel", "wait", "timed", "out", str(len(names))]
