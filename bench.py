@@ -48,7 +48,7 @@ ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out
 # was taken with (profiles/attn_sink_window_wan1.3b.md); reported only while the
 # kernel is unchanged.
 ATTN_TRAFFIC = 167.0e6         # mean of the two captured launches (166.95 MB, 167.0 MB)
-ATTN_TRAFFIC_SRC_SHA = "fb4e17ca4f14cda4"
+ATTN_TRAFFIC_SRC_SHA = "22c1b89687e2303d"
 
 
 def _peaks():
