@@ -169,6 +169,19 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
   const int li = blockIdx.x / q.n_frames;      // source layer
   const int fi = blockIdx.x % q.n_frames;      // source frame
   const int layer = q.layer0 + li;
+  const long long src0 = static_cast<long long>(blockIdx.x) * q.frame_vec;   // first vector of the frame
+  const int stride = gridDim.y * blockDim.x;
+  // the source does not depend on the counters: each thread loads its first
+  // vectors now, while thread 0 reads the counters, and then stays one
+  // iteration ahead
+  uint4 nk = make_uint4(0, 0, 0, 0), nv = make_uint4(0, 0, 0, 0);
+  {
+    const int i0 = blockIdx.y * blockDim.x + threadIdx.x;
+    if (i0 < q.frame_vec) {
+      nk = __ldg(q.src_k + src0 + i0);
+      nv = __ldg(q.src_v + src0 + i0);
+    }
+  }
   // the layer's counters, read once per block by thread 0 before the block's
   // completion count below, so the append's advance (by the last block) comes
   // after every block's read
@@ -195,8 +208,6 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
     if (reject && fi == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(q.err, KID_SCATTER | ERR_RANGE);
     slot = reject ? -1 : logical_slot(hf, ring_count, q.G, q.Ss, q.R, q.first + fi);
   }
-  const long long src0 = static_cast<long long>(blockIdx.x) * q.frame_vec;   // first vector of the frame
-  const int stride = gridDim.y * blockDim.x;
   // block-uniform trip count (slot is uniform too): every lane runs every
   // iteration, so the row-group shuffles of the quantising formats see all 32
   for (int base = slot < 0 ? q.frame_vec : blockIdx.y * blockDim.x; base < q.frame_vec; base += stride) {
@@ -210,10 +221,10 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
     const long long plane_k = (static_cast<long long>(layer) * 2 + 0) * q.H + hh;
     const long long plane_v = plane_k + q.H;
     const long long drow = static_cast<long long>(slot) * q.T + t;   // row inside a plane
-    uint4 vk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
-    if (act) {
-      vk = __ldg(q.src_k + src0 + ic);
-      vv = __ldg(q.src_v + src0 + ic);
+    const uint4 vk = nk, vv = nv;                             // this iteration's vectors (loaded ahead)
+    if (i + stride < q.frame_vec) {
+      nk = __ldg(q.src_k + src0 + i + stride);
+      nv = __ldg(q.src_v + src0 + i + stride);
     }
     store_kv_vec<FMT>(q.data, q.scales, plane_k, plane_v, q.slots, drow, q.D, vec, vk, vv, act);
   }
