@@ -74,7 +74,7 @@ typedef enum {
   LL_ERR_INVALID_ARG = 1,   /* a range, null, alignment or state check failed */
   LL_ERR_OOM = 2,           /* device allocation failed at create */
   LL_ERR_CUDA = 3,          /* a CUDA runtime/driver call or launch failed */
-  LL_ERR_UNSUPPORTED = 4,   /* valid request this build does not implement */
+  LL_ERR_UNSUPPORTED = 4,   /* valid request the library does not serve (e.g. fused call on a plain cache) */
   LL_ERR_TIMEOUT = 5        /* a bounded in-kernel wait gave up (see ll_debug_status) */
 } ll_status;
 
