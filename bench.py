@@ -47,8 +47,8 @@ ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out
 # ncu DRAM traffic of one attention launch at this shape and the kernel sources it
 # was taken with (profiles/attn_sink_window_wan1.3b.md); reported only while the
 # kernel is unchanged.
-ATTN_TRAFFIC = 167.0e6         # mean of the two captured launches (166.95 MB, 167.0 MB)
-ATTN_TRAFFIC_SRC_SHA = "22c1b89687e2303d"
+ATTN_TRAFFIC = 164.9e6         # mean of the two captured launches (166.5 MB, 163.3 MB)
+ATTN_TRAFFIC_SRC_SHA = "7f9a9c697011c607"
 
 
 def _peaks():
@@ -535,6 +535,31 @@ def run_ours(args, world, rank, local):
             "frames_seen": ll.ll_kv_cache_info(sc, 0)[0], "cache_gb": ll.ll_kv_cache_info(sc, 0)[1] / 1e9}
         sc.close()
 
+    # ---- the same step with the 30 appends batched into one launch after the
+    # attention of every layer (ll_kv_append with layer -1)
+    batched = None
+    if not args.no_fused:
+        ks_all, vs_all = torch.stack(ks), torch.stack(vs)
+
+        def bstep():
+            for l in range(L):
+                ll.ll_attn_sink_window(qs[l], ks[l], vs[l], cache, l, outs[l], stream)
+            ll.ll_kv_append(cache, -1, ks_all, vs_all, stream)
+
+        for _ in range(3):
+            bstep()
+        torch.cuda.synchronize(dev)
+        _barrier(world)
+        e0.record(stream)
+        for _ in range(args.steps):
+            bstep()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        b_ms = _max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        batched = {"ms_per_step": b_ms, "value": world * ATTN_FLOP * L / (b_ms * 1e-3) / 1e12,
+                   "launches_per_step": L + 1}
+        del ks_all, vs_all
+
     # ---- fused append: the same step with one launch per layer (attention and
     # append together) on a cache with F spare ring slots
     fused = None
@@ -637,6 +662,7 @@ def run_ours(args, world, rank, local):
         "long_rollout": sweep,
         "multishot": multishot,
         "fused_append_step": fused,
+        "batched_append_step": batched,
         "device_status": status,
     }
     if rank == 0:

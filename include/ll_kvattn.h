@@ -141,7 +141,9 @@ LL_API ll_status ll_kv_cache_create_fused(int layers, int heads, int head_dim, i
 LL_API ll_status ll_kv_shot_begin(ll_kv_cache *cache, int layer, int clear_window, ll_stream_t stream);
 
 /* ll_kv_append - store the chunk just generated in layer `layer` and evict.
- *   k_cur, v_cur: [F*T][H][D] bf16 device pointers (the chunk's K and V).
+ *   layer: 0..L-1, or -1 for every layer in one launch.
+ *   k_cur, v_cur: [F*T][H][D] bf16 device pointers (the chunk's K and V), or
+ *   [L][F*T][H][D] with layer -1.
  *   Frame f = p..p+F-1 (p = frames appended to this layer so far) goes to slot
  *   f if f < S; otherwise, if f >= p+F-W, to ring slot S + ((f-S) mod W),
  *   overwriting (evicting) the oldest window frame; other frames (only when

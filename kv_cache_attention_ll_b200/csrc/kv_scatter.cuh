@@ -229,21 +229,22 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
     store_kv_vec<FMT>(q.data, q.scales, plane_k, plane_v, q.slots, drow, q.D, vec, vk, vv, act);
   }
   if (q.mode == SCATTER_APPEND) {
-    // the last block to finish advances the counters; every block read them
-    // above, before its increment of the completion count
+    // per layer, the last of its n_frames x gridDim.y blocks to finish advances
+    // the layer's counters; every block read them above, before its increment
+    // of the layer's completion count
     __syncthreads();
     if (threadIdx.x == 0) {
       __threadfence();
-      LayerCtr *c = q.ctr + q.layer0;
-      const unsigned prev = atomicAdd(q.done + q.layer0, 1u);
-      if (prev == gridDim.x * gridDim.y - 1) {
+      LayerCtr *c = q.ctr + layer;
+      const unsigned prev = atomicAdd(q.done + layer, 1u);
+      if (prev == static_cast<unsigned>(q.n_frames) * gridDim.y - 1) {
         int fill;
         long long rc;
         append_advance(p, shot_fill, ring_count, q.G, q.Ss, q.F, &fill, &rc);
         c->p = p + q.F;
         c->shot_fill = fill;
         c->ring_count = rc;
-        q.done[q.layer0] = 0;
+        q.done[layer] = 0;
         __threadfence();
       }
     }

@@ -453,7 +453,7 @@ ll_status ll_debug_status(ll_kv_cache *c, unsigned int *word, int clear, ll_stre
 }
 
 ll_status ll_kv_append(ll_kv_cache *c, int layer, const void *k_cur, const void *v_cur, ll_stream_t stream) {
-  if (!c || layer < 0 || layer >= c->L || !k_cur || !v_cur || !aligned16(k_cur) || !aligned16(v_cur))
+  if (!c || layer < -1 || layer >= c->L || !k_cur || !v_cur || !aligned16(k_cur) || !aligned16(v_cur))
     return LL_ERR_INVALID_ARG;
   if (!on_cache_device(c)) return LL_ERR_INVALID_ARG;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -462,12 +462,15 @@ ll_status ll_kv_append(ll_kv_cache *c, int layer, const void *k_cur, const void 
     cudaGetLastError();
     return LL_ERR_CUDA;
   }
+  const int l0 = layer < 0 ? 0 : layer;
+  const int nl = layer < 0 ? c->L : 1;
   llk::ScatterParams q = scatter_base(c, k_cur, v_cur);
   q.mode = llk::SCATTER_APPEND;
-  q.layer0 = layer;
+  q.layer0 = l0;
   q.n_frames = c->F;
-  const ll_status r = launch_scatter(c, q, 1, st);
-  if (r == LL_OK) mirror_append(c, layer, cs);
+  const ll_status r = launch_scatter(c, q, nl, st);
+  if (r == LL_OK)
+    for (int l = l0; l < l0 + nl; ++l) mirror_append(c, l, cs);
   return r;
 }
 

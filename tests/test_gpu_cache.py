@@ -159,3 +159,33 @@ def test_invalid_recache_ranges_are_rejected():
             ll.ll_kv_append(cache, 0, buf.data_ptr() + 2, buf.data_ptr())
     finally:
         cache.close()
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8", "nvfp4"])
+def test_append_of_all_layers_in_one_launch(kv_dtype):
+    """ll_kv_append(cache, -1, k[L], v[L]) stores every layer's chunk in one
+    launch and advances every layer's counters: the cache bytes equal the
+    oracle's per-layer appends, with shot starts in between."""
+    import torch
+    from gpu_util import to_dev
+    ll = _ll()
+    L, H, D, T, F, G, Ss, W = 3, 2, 128, 20, 3, 2, 1, 4
+    model = CacheModel(L, H, D, T, F, G, W, kv_dtype, shot_sink_frames=Ss)
+    cache = ll.ll_kv_cache_create_multishot(L, H, D, T, F, G, Ss, W, kv_dtype)
+    try:
+        for c in range(7):
+            if c in (3, 5):
+                ll.ll_kv_shot_begin(cache, -1, c == 5)
+                model.shot_begin(-1, c == 5)
+            ks = np.stack([chunk_qkv(400, l, c, F * T, H, D)[1] for l in range(L)])
+            vs = np.stack([chunk_qkv(400, l, c, F * T, H, D)[2] for l in range(L)])
+            ll.ll_kv_append(cache, -1, to_dev(ks), to_dev(vs))
+            for l in range(L):
+                model.append(l, ks[l], vs[l])
+            torch.cuda.synchronize()
+            for l in range(L):
+                assert ll.ll_kv_cache_export(cache, l) == model.export(l), f"chunk {c} layer {l}"
+                assert ll.ll_kv_cache_info(cache, l)[0] == (c + 1) * F
+        assert ll.ll_debug_status(cache) == 0
+    finally:
+        cache.close()
