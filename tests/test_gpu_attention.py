@@ -79,6 +79,18 @@ def test_wan_shape_sampled_rows():
     assert len(res) == 4
 
 
+def test_full_causal_largest_history_sampled_rows():
+    """The longest history the pages measure: their full-causal comparison runs
+    40 chunks (117 latent frames of 1560 tokens) with every earlier frame
+    visible (sink 3 + window 114). Chunk 39 attends 187200 keys (117 cached
+    frames and its own 3), 8 times the steady-state sink + window count. Two
+    heads of the Wan frame size (heads are independent; the key count is what
+    grows); chunk 13 (42 cached frames) and chunk 39, sampled rows with the
+    ragged last query tile."""
+    res = _rollout(41, H=2, D=128, T=1560, F=3, S=3, W=114, n_chunks=40, check={13, 39}, rows_per_head=256)
+    assert len(res) == 2
+
+
 def test_large_logits_rescale_path():
     """Q and K scaled by 4 so that logits span tens of units: exercises the lazy
     rescale of O. The softmax is peaked here, so the max-abs bound is the one
