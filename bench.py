@@ -288,9 +288,14 @@ def _library_context(ll, torch, cache, qs, ks, vs, stream, dev):
                     "cudnn_with_gather": "torch.cat of the held K/V and the own chunk, then cuDNN"}}
     try:
         with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            # one launch of each in an NVTX range, so that a profiler can select
+            # exactly this pair (ncu --nvtx --nvtx-include "ll_vs_cudnn/")
+            torch.cuda.nvtx.range_push("ll_vs_cudnn")
             ours(0, ours_out)
+            torch.cuda.synchronize(dev)
             ref = lib(0)
             torch.cuda.synchronize(dev)
+            torch.cuda.nvtx.range_pop()
             a = ours_out.float()
             b = ref[0].permute(1, 0, 2).float()
             res["layer0_max_abs_diff"] = (a - b).abs().max().item()
