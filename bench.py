@@ -38,6 +38,9 @@ TQ = F * T
 NK = (S + W + F) * T                       # visible keys in steady state: 23400
 ATTN_FLOP = 4.0 * TQ * NK * D * H          # per layer: QK^T and PV over visible keys only
 APPEND_BYTES = 2 * 2 * TQ * H * D * 2      # K and V, read + write
+# bytes per cached (token, head) row of a quantised cache: FP8 codes + one fp32
+# scale; NVFP4 codes (two per byte) + one E4M3 scale per 16 values
+QUANT_ROW_BYTES = {"fp8": D + 4, "nvfp4": D // 2 + D // 16}
 
 
 def recache_bytes(layers: int) -> int:
@@ -545,8 +548,23 @@ def run_ours(args, world, rank, local):
             q_ms = e0.elapsed_time(e1) / args.quant_steps
             q_attn = statistics.mean(a.elapsed_time(b) for ev in qev for a, b in ev)
             qbytes = ll.ll_kv_cache_info(qc, 0)[1]
+            # append alone, quantising on write, timed like the bf16 append:
+            # reads the bf16 chunk, writes codes and scales
+            qa = []
+            for _ in range(max(3, args.steps)):
+                e0.record(stream)
+                for l in range(L):
+                    ll.ll_kv_append(qc, l, ks[l], vs[l], stream)
+                e1.record(stream)
+                e1.synchronize()
+                qa.append(e0.elapsed_time(e1) / L)
+            qa_ms = statistics.median(qa)
+            qa_bytes = 2 * TQ * H * D * 2 + 2 * TQ * H * QUANT_ROW_BYTES[kvd]
             quant[kvd] = {"ms_per_step": q_ms, "value": ATTN_FLOP * L / (q_ms * 1e-3) / 1e12,
                           "attn_launch_ms": q_attn, "attn_tflops": ATTN_FLOP / (q_attn * 1e-3) / 1e12,
+                          "append": {"ms_per_layer": qa_ms, "bytes": qa_bytes,
+                                     "gbs": qa_bytes / (qa_ms * 1e-3) / 1e9,
+                                     "frac_hbm": qa_bytes / (qa_ms * 1e-3) / 1e9 / peak_gbs},
                           "cache_gb": qbytes / 1e9, "cache_gb_bf16": cache_bytes_bf16 / 1e9,
                           "device_status": ll.ll_debug_status(qc)}
             qc.close()
