@@ -207,6 +207,28 @@ def cpu_oracle_sample(seconds_target: float = 12.0, n_rows: int | None = None):
     return flop / dt / 1e12, desc, threads, n_rows
 
 
+def cpu_oracle_config0():
+    """The whole tiny configuration on the CPU oracle: 2 heads, head_dim 64, 16
+    tokens per frame, chunk 3, sink 3, window 6, attention of all 8 chunks
+    (every row; input generation not timed). Returns seconds, work and rows."""
+    import numpy as np
+    import oracle
+    from seeded_inputs import chunk_qkv
+    h0, d0, t0, f0, s0, w0, n = 2, 64, 16, 3, 3, 6, 8
+    chunks = [chunk_qkv(0, 0, c, f0 * t0, h0, d0) for c in range(n)]
+    flop = 0.0
+    start = time.perf_counter()
+    for c in range(n):
+        kh = np.concatenate([x[1] for x in chunks[:c + 1]])
+        vh = np.concatenate([x[2] for x in chunks[:c + 1]])
+        oracle.sink_window_attention(chunks[c][0], kh, vh, c, s0, w0, f0, t0)
+        p = c * f0
+        keys = (min(p, s0) + min(w0, max(0, p - s0)) + f0) * t0
+        flop += 4.0 * f0 * t0 * keys * d0 * h0
+    dt = time.perf_counter() - start
+    return {"workload": "2 heads, head_dim 64, 16 tokens/frame, chunk 3, sink 3, window 6, 8 chunks, all rows",
+            "seconds": dt, "tflop": flop / 1e12}
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -751,7 +773,8 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, threads, _ = cpu_oracle_sample()
-        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+               "tiny_config_full_run": cpu_oracle_config0()}
 
     status = ll.ll_debug_status(cache)
     cache.close()

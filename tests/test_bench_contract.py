@@ -52,3 +52,13 @@ def test_recorded_traffic_matches_the_kernel_sources():
         # a launch cannot move less than its minimum bytes by much (L2 hits aside)
         # and wasted re-reads would show as far more
         assert 0.8 * bench.ATTN_MIN_BYTES < bench.ATTN_TRAFFIC < 1.5 * bench.ATTN_MIN_BYTES
+
+
+def test_tiny_configuration_oracle_run():
+    """The CPU baseline also times the whole tiny configuration: 8 chunks whose
+    visible keys grow 48, 96, 144, then 192 (sink 3 + window 6 + own 3 frames
+    of 16 tokens) for the last five."""
+    r = bench.cpu_oracle_config0()
+    keys = 48 + 96 + 144 + 5 * 192
+    assert r["tflop"] * 1e12 == pytest.approx(4 * 48 * keys * 64 * 2, rel=1e-12)
+    assert 0 < r["seconds"] < 30
