@@ -41,6 +41,9 @@ APPEND_BYTES = 2 * 2 * TQ * H * D * 2      # K and V, read + write
 # bytes per cached (token, head) row of a quantised cache: FP8 codes + one fp32
 # scale; NVFP4 codes (two per byte) + one E4M3 scale per 16 values
 QUANT_ROW_BYTES = {"fp8": D + 4, "nvfp4": D // 2 + D // 16}
+# datasheet dense bf16 tensor throughput of one B200 (the sparse figure is twice
+# this); reported beside the measured peaks, labelled as the datasheet's
+DATASHEET_BF16_DENSE_TFLOPS = 2250.0
 
 
 def recache_bytes(layers: int) -> int:
@@ -791,6 +794,7 @@ def run_ours(args, world, rank, local):
                    "parallelism": f"replicas x{world} (independent streams)"},
         "pct_bf16_peak": value / peak_tf,
         "pct_bf16_peak_sustained": value / peak_tf_sust,
+        "pct_bf16_datasheet_dense": value / DATASHEET_BF16_DENSE_TFLOPS,
         "latent_frames_per_s": world * F / (ms_step * 1e-3),
         # the attention launches are timed inside the long timed region (seconds
         # of steps under the power cap), so the sustained GEMM figure is the peak
@@ -798,6 +802,7 @@ def run_ours(args, world, rank, local):
                      "frac": attn_tf / peak_tf_sust, "traffic": traffic,
                      "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a long step)",
                      "frac_of_burst": attn_tf / peak_tf, "burst_peak": peak_tf,
+                     "frac_of_datasheet_dense": attn_tf / DATASHEET_BF16_DENSE_TFLOPS,
                      "kernel": "attn_sink_window_kernel<128>", "launch_ms": attn_avg,
                      "algorithmic_flop_per_launch": ATTN_FLOP, "min_bytes_per_launch": ATTN_MIN_BYTES},
         "append": {"ms_per_layer": app_ms, "gbs": APPEND_BYTES / (app_ms * 1e-3) / 1e9,

@@ -62,3 +62,8 @@ def test_tiny_configuration_oracle_run():
     keys = 48 + 96 + 144 + 5 * 192
     assert r["tflop"] * 1e12 == pytest.approx(4 * 48 * keys * 64 * 2, rel=1e-12)
     assert 0 < r["seconds"] < 30
+
+
+def test_datasheet_figure_is_the_dense_one():
+    # 2.25 PFLOP/s dense bf16; the 4.5 PFLOP/s figure assumes 2:4 sparsity
+    assert bench.DATASHEET_BF16_DENSE_TFLOPS == 2250.0
