@@ -8,8 +8,12 @@ used. The pages give no rounding or scaling details; the readings taken here:
 
 FP8 (E4M3, per (token, head) row of D values, one fp32 scale per row)
   1. amax  = max |x|                        (exact)
-  2. scale = amax / 448   (fp32 division);  scale = 1 if amax == 0
-  3. inv   = 1 / scale    (fp32 division)
+  2. scale = max(amax / 448, 2^-126)   (fp32 division);  scale = 1 if amax == 0
+     The floor is the smallest normal fp32 value: below it 1 / scale would
+     overflow to infinity (a row whose maximum is under 448 * 2^-126, about
+     2^-117, would otherwise turn its zeros into NaN codes and its other
+     values into saturated ones). Rows at or above that maximum are unchanged.
+  3. inv   = 1 / scale    (fp32 division; finite, at most 2^126)
   4. code  = E4M3(x * inv)   fp32 product, then round-to-nearest-even into E4M3
              with saturation to +-448 (no NaN is ever produced)
   dequantised value = E4M3 value * scale
@@ -35,6 +39,7 @@ import numpy as np
 
 E4M3_MAX = 448.0
 E2M1_MAX = 6.0
+FP8_MIN_SCALE = 2.0 ** -126     # smallest normal fp32: keeps 1 / scale finite
 
 
 def e4m3_value(code: int) -> float:
@@ -100,7 +105,8 @@ def fp8_quantize_rows(x_bits: np.ndarray):
     """bf16 rows [..., D] (uint16 bits) -> (codes uint8 [..., D], scales float32 [...])."""
     x = (np.asarray(x_bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
     amax = np.max(np.abs(x), axis=-1)                                  # fp32, exact
-    scale = np.where(amax == 0, np.float32(1.0), amax / np.float32(E4M3_MAX)).astype(np.float32)
+    scale = np.maximum(amax / np.float32(E4M3_MAX), np.float32(FP8_MIN_SCALE)).astype(np.float32)
+    scale = np.where(amax == 0, np.float32(1.0), scale).astype(np.float32)
     inv = (np.float32(1.0) / scale).astype(np.float32)
     y = (x * inv[..., None]).astype(np.float32)                        # fp32 products
     return e4m3_encode(y), scale

@@ -91,6 +91,40 @@ def test_fp8_zero_row_and_sign():
     assert codes[1, 0, 3] == 0xFE and sc[1, 0] == np.float32(2.0) / np.float32(448)
 
 
+def test_fp8_tiny_rows_use_the_floor_scale():
+    """Rows whose maximum is below 448 * 2^-126 take the floor scale 2^-126, so
+    that 1/scale = 2^126 stays finite. Hand-derived: a row holding only the
+    smallest positive bf16 subnormal 2^-133 has x * 2^126 = 2^-7 = 4 * 2^-9,
+    the E4M3 subnormal with mantissa 4 (code 0x04); its zeros stay code 0x00;
+    at exactly 448 * 2^-126 the division gives the floor itself."""
+    y = np.zeros((3, 16), dtype=np.uint16)
+    y[0, 2] = 0x0001                                     # 2^-133
+    y[1, 0] = 0x8001                                     # -2^-133
+    y[2, 5] = f32_to_bf16_bits(np.array([448.0 * 2.0 ** -126], dtype=np.float32))[0]
+    codes, sc = quant.fp8_quantize_rows(y)
+    assert sc.view(np.uint32).tolist() == [0x00800000] * 3
+    assert codes[0, 2] == 0x04 and codes[1, 0] == 0x84 and codes[2, 5] == 0x7E
+    assert int(np.count_nonzero(codes)) == 3
+
+
+def test_fp8_every_bf16_row_maximum_gives_finite_codes():
+    """Every finite bf16 value as the only non-zero element of a row, next to a
+    zero: no NaN code (S.1111.111) ever appears, the scale is finite and
+    positive, and the value comes back within the E4M3 bound (half a step:
+    2^-4 relative for normals, 2^-10 * scale for subnormals)."""
+    p = np.arange(1 << 16, dtype=np.uint32)
+    p = p[((p >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    x = np.zeros((len(p), 2), dtype=np.uint16)
+    x[:, 0] = p
+    codes, sc = quant.fp8_quantize_rows(x)
+    assert not np.any((codes & 0x7F) == 0x7F)
+    assert np.all(np.isfinite(sc)) and np.all(sc > 0)
+    xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    err = np.abs(quant.fp8_dequantize_rows(codes, sc) - xf)
+    bound = np.maximum(np.abs(xf) * 2.0 ** -4, sc[:, None].astype(np.float64) * 2.0 ** -10)
+    assert np.all(err <= bound * (1 + 1e-6))
+
+
 def test_nvfp4_blocks_error_bound_and_packing():
     x = bf16_normal(mix_seed(9, 9), (200, 3, 64))
     packed, sb = quant.nvfp4_quantize_rows(x)
