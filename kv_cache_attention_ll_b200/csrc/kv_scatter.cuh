@@ -113,7 +113,9 @@ __device__ __forceinline__ void store_kv_vec(uint8_t *data, uint8_t *scales, lon
       *dv = vv;
     }
   } else if constexpr (FMT == FMT_FP8) {
-    // per (token, head) row: scale = amax/448 (1 if amax == 0), codes = E4M3(x * (1/scale))
+    // per (token, head) row: scale = max(amax/448, 2^-126) (1 if amax == 0),
+    // codes = E4M3(x * (1/scale)); the floor (smallest normal fp32) keeps 1/scale
+    // finite for rows whose maximum is below 448 * 2^-126
 #pragma unroll
     for (int kv = 0; kv < 2; ++kv) {
       float x[8];
@@ -122,7 +124,7 @@ __device__ __forceinline__ void store_kv_vec(uint8_t *data, uint8_t *scales, lon
 #pragma unroll
       for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
       for (int o = 1; o < vpr; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const float scale = amax == 0.f ? 1.0f : __fdiv_rn(amax, 448.0f);
+      const float scale = amax == 0.f ? 1.0f : fmaxf(__fdiv_rn(amax, 448.0f), 0x1p-126f);
       const float inv = __fdiv_rn(1.0f, scale);
       float y[8];
 #pragma unroll
