@@ -244,8 +244,8 @@ LL_API ll_status ll_kv_cache_export(const ll_kv_cache *cache, int layer, void *h
                              ll_stream_t stream);
 
 /* ll_attn_sink_window_noalloc - the attention of ll_attn_sink_window over a
- *   quantised cache layer (FP8 or NVFP4) held in caller memory, performing no
- *   device allocation at all. The pages have no counterpart: this entry point
+ *   quantised single-shot cache layer (FP8 or NVFP4) held in caller memory,
+ *   performing no device allocation at all. The pages have no counterpart: this entry point
  *   exists for callers that cannot call cudaMalloc, for example code whose
  *   device memory is owned entirely by a host framework's pool (a serving
  *   engine that reserves all memory up front and forbids libraries from
@@ -255,10 +255,14 @@ LL_API ll_status ll_kv_cache_export(const ll_kv_cache *cache, int layer, void *h
  *   layer_codes [2][H][(S+W)*T][row bytes] (K planes, then V planes; row bytes
  *   D for FP8, D/2 for NVFP4) and layer_scales [2][H][(S+W)*T][...] (fp32 per
  *   row for FP8, D/16 E4M3 bytes per row for NVFP4) - the layout that
- *   ll_kv_cache_export writes for one layer (data part, then scale part);
- *   frames_seen = frames appended to this layer so far (p). Output: out
- *   [F*T][H][D] bf16. Results equal those of ll_attn_sink_window on a cache
- *   holding the same bytes.
+ *   ll_kv_cache_export writes for one layer (data part, then scale part) of a
+ *   cache made by ll_kv_cache_create (S + W slots per plane, the window ring
+ *   starting at slot S) on which ll_kv_shot_begin was never called;
+ *   frames_seen = that layer's own frame counter p (frames appended to it so
+ *   far). Layers of multi-shot or fused caches, or of a cache after a shot
+ *   start, have another slot layout and are not accepted (their results would
+ *   be wrong). Output: out [F*T][H][D] bf16. Results equal those of
+ *   ll_attn_sink_window on a cache holding the same bytes.
  *   Scratch: the dequantised bf16 view of the layer, 2*H*(S+W)*T*D*2 bytes,
  *   lives in a file-scope device array of LL_NOALLOC_SCRATCH_BYTES that every
  *   GPU loading the library holds until exit. Larger geometries are rejected
@@ -267,7 +271,9 @@ LL_API ll_status ll_kv_cache_export(const ll_kv_cache *cache, int layer, void *h
  *   GPU (different streams, or different host threads, on one device) race:
  *   order them. The first call on a device looks up the array's device
  *   address (once per device, with that device current); make that first call
- *   before any stream capture. No status word is written by this path.     */
+ *   before any stream capture. A bounded in-kernel wait that gives up (the
+ *   output is then incomplete) is recorded in this path's own device status
+ *   word, read with ll_noalloc_debug_status.                                */
 #define LL_NOALLOC_SCRATCH_BYTES (16u << 20)
 LL_API ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const void *v_cur,
                                              const void *layer_codes, const void *layer_scales,
@@ -275,6 +281,13 @@ LL_API ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, c
                                              int tokens_per_frame, int frames_per_chunk, int sink_frames,
                                              int window_frames, long long frames_seen, void *out,
                                              ll_stream_t stream);
+
+/* Status word of ll_attn_sink_window_noalloc's kernels on the current device
+ * (one per device, shared by every call of that entry point): as for
+ * ll_debug_status, reading synchronises `stream`, `clear` resets it to 0, and
+ * the return value is LL_ERR_TIMEOUT if a bounded wait gave up, LL_OK for 0.
+ * Allocates nothing.                                                        */
+LL_API ll_status ll_noalloc_debug_status(unsigned int *word, int clear, ll_stream_t stream);
 
 /* Device-side status word of the cache's kernels: 0 = fine; otherwise OR-ed
  * flags, reasons in the low byte (1 = a bounded in-kernel wait gave up,

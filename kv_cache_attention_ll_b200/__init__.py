@@ -41,6 +41,7 @@ _sig = {
     "ll_debug_status": (_i, [_vp, ctypes.POINTER(ctypes.c_uint), _i, _vp]),
     "ll_attn_sink_window_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _ll, _vp, _vp]),
     "ll_debug_wait_selftest": (_i, [_vp, _vp]),
+    "ll_noalloc_debug_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i, _vp]),
     "ll_kv_cache_create_multishot": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
     "ll_kv_shot_begin": (_i, [_vp, _i, _i, _vp]),
     "ll_kv_cache_held": (_i, [_vp, _i, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
@@ -237,12 +238,22 @@ def ll_attn_sink_window_noalloc(q, k_cur, v_cur, layer_codes, layer_scales, kv_d
     """Attention over one quantised cache layer held in caller memory, with no
     device allocation (the scratch is a static device array of the library).
     layer_codes / layer_scales: device buffers (uint8 tensors or pointers) in
-    the layout ll_kv_cache_export writes for one layer."""
+    the layout ll_kv_cache_export writes for one layer of a single-shot cache
+    (ll_kv_cache_create, no shot start); frames_seen: that layer's counter."""
     dt = _DTYPES[kv_dtype] if isinstance(kv_dtype, str) else int(kv_dtype)
     _check(_lib.ll_attn_sink_window_noalloc(_ptr(q), _ptr(k_cur), _ptr(v_cur), _raw_ptr(layer_codes),
                                             _raw_ptr(layer_scales), dt, heads, head_dim, tokens_per_frame,
                                             frames_per_chunk, sink_frames, window_frames, frames_seen, _ptr(out),
                                             _stream(stream)), "ll_attn_sink_window_noalloc")
+
+
+def ll_noalloc_debug_status(clear: bool = False, stream=None) -> int:
+    """Status word of ll_attn_sink_window_noalloc's kernels on the current device (0 = fine)."""
+    w = ctypes.c_uint()
+    st = _lib.ll_noalloc_debug_status(ctypes.byref(w), int(clear), _stream(stream))
+    if st not in (LL_OK, LL_ERR_TIMEOUT, LL_ERR_INVALID_ARG):
+        _check(st, "ll_noalloc_debug_status")
+    return w.value
 
 
 def _raw_ptr(x) -> int:

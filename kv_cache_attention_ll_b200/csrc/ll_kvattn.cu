@@ -658,25 +658,34 @@ extern "C" ll_status ll_debug_wait_selftest(ll_kv_cache *c, ll_stream_t stream) 
 // per device with cudaGetSymbolAddress (with that device current) and passed
 // to the kernels.
 static __device__ __align__(256) uint8_t g_noalloc_view[LL_NOALLOC_SCRATCH_BYTES];
+// the status word of this path's kernels (the cache path keeps its own in the
+// cache allocation): a bounded wait that gives up is recorded here
+static __device__ __align__(256) unsigned g_noalloc_status;
 
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void *g_noalloc_addr[kMaxDevices] = {};
+unsigned *g_noalloc_status_addr[kMaxDevices] = {};
 
-// device address of g_noalloc_view on the current device (nullptr on failure)
-void *noalloc_scratch(int dev) {
-  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+// device addresses of g_noalloc_view and g_noalloc_status on device `dev`,
+// which must be current (false on failure)
+bool noalloc_scratch(int dev, void **view, unsigned **status) {
+  if (dev < 0 || dev >= kMaxDevices) return false;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
   if (!g_noalloc_addr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_view) != cudaSuccess) {
+    void *v = nullptr, *st = nullptr;
+    if (cudaGetSymbolAddress(&v, g_noalloc_view) != cudaSuccess ||
+        cudaGetSymbolAddress(&st, g_noalloc_status) != cudaSuccess) {
       cudaGetLastError();
-      return nullptr;
+      return false;
     }
-    g_noalloc_addr[dev] = ptr;
+    g_noalloc_status_addr[dev] = static_cast<unsigned *>(st);
+    g_noalloc_addr[dev] = v;
   }
-  return g_noalloc_addr[dev];
+  *view = g_noalloc_addr[dev];
+  *status = g_noalloc_status_addr[dev];
+  return true;
 }
 }  // namespace
 
@@ -704,8 +713,10 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
-  uint8_t *view = static_cast<uint8_t *>(noalloc_scratch(dev));
-  if (!view) return LL_ERR_CUDA;
+  void *view_ptr = nullptr;
+  unsigned *status = nullptr;
+  if (!noalloc_scratch(dev, &view_ptr, &status)) return LL_ERR_CUDA;
+  uint8_t *view = static_cast<uint8_t *>(view_ptr);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
   // held context, as for a cache whose layer counter is frames_seen
@@ -757,7 +768,7 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
                    static_cast<uint64_t>(slots) * head_dim * 2, 64, kKeyTile, 1))
     return LL_ERR_CUDA;
   prm.out = static_cast<__nv_bfloat16 *>(out);
-  prm.err = nullptr;
+  prm.err = status;
   prm.H = heads;
   prm.Tq = Tq;
   prm.n_cache = n_cache;
@@ -767,6 +778,23 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
   const int grid = prm.num_q_tiles * heads;
   return head_dim == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
+}
+
+ll_status ll_noalloc_debug_status(unsigned int *word, int clear, ll_stream_t stream) {
+  if (!word) return LL_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
+  void *view = nullptr;
+  unsigned *status = nullptr;
+  if (!noalloc_scratch(dev, &view, &status)) return LL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned w = 0;
+  if (cudaMemcpyAsync(&w, status, sizeof(w), cudaMemcpyDeviceToHost, s) != cudaSuccess) return LL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LL_ERR_CUDA;
+  if (clear && cudaMemsetAsync(status, 0, sizeof(unsigned), s) != cudaSuccess) return LL_ERR_CUDA;
+  *word = w;
+  if (w & llk::ERR_WAIT_TIMEOUT) return LL_ERR_TIMEOUT;
+  return w ? LL_ERR_INVALID_ARG : LL_OK;
 }
 
 }  // extern "C"

@@ -98,11 +98,12 @@ def test_large_logits_rescale_path():
     _rollout(21, H=2, D=128, T=64, F=3, S=3, W=6, n_chunks=6, check={2, 5}, qk_scale=4.0)
 
 
-def test_large_max_jump_recompute_path():
+def test_large_max_jump_rescale_path():
     """The chunk's own keys scaled by 40: its tiles come after the cache tiles and
-    raise the row max by far more than 2^64 over the running reference, which
-    forces the exact recompute of those tiles (and a later O rescale). The
-    softmax is peaked, so the derived bf16 bound applies."""
+    raise a row's maximum logit far above the running reference maximum (much
+    more than the lazy-rescale threshold of 8 in log2 units), so the reference
+    moves up and the partial output and row sum are rescaled before those
+    tiles are added. The softmax is peaked, so the derived bf16 bound applies."""
     import torch
     import kv_cache_attention_ll_b200 as ll
     from gpu_util import to_dev, dev_to_f64, assert_attn_close_derived

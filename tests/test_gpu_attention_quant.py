@@ -1,7 +1,9 @@
 """GPU parity of ll_attn_sink_window on FP8 and NVFP4 caches.
 
 The library quantises on append (bit-exact against the oracle, see
-test_gpu_cache.py) and dequantises inside the attention kernel. The oracle
+test_gpu_cache.py). Each attention call first converts the layer's held codes
+into a bf16 view of the cache (a separate pass of the same call), and the
+attention kernel reads that view. The oracle
 attends over the exactly dequantised held frames (E4M3 code x fp32 row scale,
 or E2M1 code x E4M3 block scale, in fp64) plus the chunk's own bf16 K/V, with
 its explicit sink + window + block-causal mask.
