@@ -8,15 +8,21 @@ used. The pages give no rounding or scaling details; the readings taken here:
 
 FP8 (E4M3, per (token, head) row of D values, one fp32 scale per row)
   1. amax  = max |x|                        (exact)
-  2. scale = max(amax / 448, 2^-126)   (fp32 division);  scale = 1 if amax == 0
-     The floor is the smallest normal fp32 value: below it 1 / scale would
-     overflow to infinity (a row whose maximum is under 448 * 2^-126, about
-     2^-117, would otherwise turn its zeros into NaN codes and its other
-     values into saturated ones). Rows at or above that maximum are unchanged.
-  3. inv   = 1 / scale    (fp32 division; finite, at most 2^126)
-  4. code  = E4M3(x * inv)   fp32 product, then round-to-nearest-even into E4M3
-             with saturation to +-448 (no NaN is ever produced)
-  dequantised value = E4M3 value * scale
+  2. scale = the smallest power of two s with amax <= 448 * s, but at least
+     2^-124;  scale = 1 if amax == 0.
+     A power-of-two scale keeps every step exact: x / scale is an exact fp32
+     value (no rounding before the E4M3 rounding; only quotients far below
+     the smallest E4M3 step can underflow, and they encode as zero either
+     way), and every dequantised
+     value, E4M3 value * scale, has at most 4 significant bits and lies at or
+     above 2^-133, so it is exact in bf16 (the floor 2^-124 guarantees the
+     latter and keeps 1 / scale finite). The row maximum lands in (224, 448],
+     so E4M3's 3-bit relative precision is kept for every value but the
+     lowest binade of the row's range.
+  3. inv   = 1 / scale    (exact, a power of two)
+  4. code  = E4M3(x * inv)   fp32 product (exact, as above), then round-to-nearest-even
+             into E4M3 with saturation to +-448 (no NaN is ever produced)
+  dequantised value = E4M3 value * scale (exact in bf16)
 
 NVFP4 (E2M1 values, 16-element blocks along D, E4M3 block scale)
   1. amax = max |x| over the block
@@ -39,7 +45,7 @@ import numpy as np
 
 E4M3_MAX = 448.0
 E2M1_MAX = 6.0
-FP8_MIN_SCALE = 2.0 ** -126     # smallest normal fp32: keeps 1 / scale finite
+FP8_MIN_SCALE_LOG2 = -124      # scale floor: dequantised values stay exact in bf16
 
 
 def e4m3_value(code: int) -> float:
@@ -104,11 +110,16 @@ def e2m1_encode(y) -> np.ndarray:
 def fp8_quantize_rows(x_bits: np.ndarray):
     """bf16 rows [..., D] (uint16 bits) -> (codes uint8 [..., D], scales float32 [...])."""
     x = (np.asarray(x_bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
-    amax = np.max(np.abs(x), axis=-1)                                  # fp32, exact
-    scale = np.maximum(amax / np.float32(E4M3_MAX), np.float32(FP8_MIN_SCALE)).astype(np.float32)
-    scale = np.where(amax == 0, np.float32(1.0), scale).astype(np.float32)
-    inv = (np.float32(1.0) / scale).astype(np.float32)
-    y = (x * inv[..., None]).astype(np.float32)                        # fp32 products
+    amax = np.max(np.abs(x), axis=-1).astype(np.float64)               # exact
+    # smallest k with amax <= 448 * 2^k: amax / 448 and its log2 are exact in
+    # fp64 whenever the result is an integer (amax = 7 * 2^j for bf16 inputs),
+    # and otherwise nowhere near one
+    with np.errstate(divide="ignore"):
+        k = np.ceil(np.log2(amax / E4M3_MAX))
+    k = np.where(amax == 0, 0.0, np.maximum(k, FP8_MIN_SCALE_LOG2))
+    scale = np.exp2(k).astype(np.float32)                              # powers of two: exact
+    inv = np.exp2(-k).astype(np.float32)
+    y = (x * inv[..., None]).astype(np.float32)                        # fp32 products (exact)
     return e4m3_encode(y), scale
 
 

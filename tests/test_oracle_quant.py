@@ -73,14 +73,35 @@ def test_fp8_rows_error_bound_and_scale():
     codes, sc = quant.fp8_quantize_rows(x)
     xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     amax = np.abs(xf).max(-1)
-    np.testing.assert_array_equal(sc, (amax.astype(np.float32) / np.float32(448)).astype(np.float32))
+    # the scale is a power of two with amax / 448 <= scale < 2 * amax / 448
+    m, _ = np.frexp(sc.astype(np.float64))
+    assert np.all(m == 0.5)
+    assert np.all(amax <= 448 * sc) and np.all(448 * sc < 2 * amax)
     deq = quant.fp8_dequantize_rows(codes, sc)
     # E4M3 has 3 fraction bits: relative error <= 2^-4 for normals, absolute <= 2^-10 * scale below
     err = np.abs(deq - xf)
     bound = np.maximum(np.abs(xf) * 2.0 ** -4, sc[..., None].astype(np.float64) * 2.0 ** -10)
     assert np.all(err <= bound * (1 + 1e-6))
-    # the row maximum maps to +-448 exactly or within one step
-    assert np.all(np.abs(quant.E4M3_TABLE[codes]).max(-1) >= 416)
+    # the row maximum lands in (224, 448] before rounding, so its code is at least 224
+    assert np.all(np.abs(quant.E4M3_TABLE[codes]).max(-1) >= 224)
+    # every dequantised value is exact in bf16 (at most 8 significant bits, in range)
+    d32 = deq.astype(np.float32)
+    assert np.all(d32.astype(np.float64) == deq)
+    assert np.all((d32.view(np.uint32) & 0xFFFF) == 0)
+
+
+def test_fp8_scale_hand_derived_cases():
+    """Hand-derived: a row with maximum 448 has scale 1 and keeps its values
+    (448 -> 0x7E, -1 -> 0xB8); 450 (exact in bf16) needs scale 2: 450/2 = 225
+    rounds to the E4M3 value 224 (0x76), 3/2 = 1.5 (0x3C); a maximum of 1
+    gives scale 2^-8 (1/448 lies between 2^-9 and 2^-8), so 1 -> 256 (0x78)
+    and 0.5 -> 128 (0x70); a maximum of exactly 7 * 2^-6 = 448 * 2^-12 gives
+    scale 2^-12 exactly and the code 448 (0x7E)."""
+    vals = [[448.0, -1.0], [450.0, 3.0], [1.0, 0.5], [7 * 2.0 ** -6, 0.0]]
+    y = np.array([f32_to_bf16_bits(np.array(v, dtype=np.float32)) for v in vals], dtype=np.uint16)
+    codes, sc = quant.fp8_quantize_rows(y)
+    assert sc.tolist() == [1.0, 2.0, 2.0 ** -8, 2.0 ** -12]
+    assert codes.tolist() == [[0x7E, 0xB8], [0x76, 0x3C], [0x78, 0x70], [0x7E, 0x00]]
 
 
 def test_fp8_zero_row_and_sign():
@@ -88,30 +109,33 @@ def test_fp8_zero_row_and_sign():
     x[1, 0, 3] = f32_to_bf16_bits(np.array([-2.0], dtype=np.float32))[0]
     codes, sc = quant.fp8_quantize_rows(x)
     assert sc[0, 0] == 1.0 and not codes[0].any()
-    assert codes[1, 0, 3] == 0xFE and sc[1, 0] == np.float32(2.0) / np.float32(448)
+    # amax 2: scale 2^-7 (2/448 lies between 2^-8 and 2^-7), -2 * 128 = -256 -> 0xF8
+    assert codes[1, 0, 3] == 0xF8 and sc[1, 0] == np.float32(2.0 ** -7)
 
 
 def test_fp8_tiny_rows_use_the_floor_scale():
-    """Rows whose maximum is below 448 * 2^-126 take the floor scale 2^-126, so
-    that 1/scale = 2^126 stays finite. Hand-derived: a row holding only the
-    smallest positive bf16 subnormal 2^-133 has x * 2^126 = 2^-7 = 4 * 2^-9,
-    the E4M3 subnormal with mantissa 4 (code 0x04); its zeros stay code 0x00;
-    at exactly 448 * 2^-126 the division gives the floor itself."""
+    """Rows whose maximum is below 448 * 2^-124 take the floor scale 2^-124.
+    Hand-derived: a row holding only the smallest positive bf16 subnormal
+    2^-133 has x * 2^124 = 2^-9, the smallest E4M3 subnormal (code 0x01);
+    its zeros stay code 0x00; at exactly 448 * 2^-124 the maximum gets the
+    floor itself and the code 448 (0x7E)."""
     y = np.zeros((3, 16), dtype=np.uint16)
     y[0, 2] = 0x0001                                     # 2^-133
     y[1, 0] = 0x8001                                     # -2^-133
-    y[2, 5] = f32_to_bf16_bits(np.array([448.0 * 2.0 ** -126], dtype=np.float32))[0]
+    y[2, 5] = f32_to_bf16_bits(np.array([448.0 * 2.0 ** -124], dtype=np.float32))[0]
     codes, sc = quant.fp8_quantize_rows(y)
-    assert sc.view(np.uint32).tolist() == [0x00800000] * 3
-    assert codes[0, 2] == 0x04 and codes[1, 0] == 0x84 and codes[2, 5] == 0x7E
+    assert sc.view(np.uint32).tolist() == [0x01800000] * 3
+    assert codes[0, 2] == 0x01 and codes[1, 0] == 0x81 and codes[2, 5] == 0x7E
     assert int(np.count_nonzero(codes)) == 3
 
 
 def test_fp8_every_bf16_row_maximum_gives_finite_codes():
     """Every finite bf16 value as the only non-zero element of a row, next to a
-    zero: no NaN code (S.1111.111) ever appears, the scale is finite and
-    positive, and the value comes back within the E4M3 bound (half a step:
-    2^-4 relative for normals, 2^-10 * scale for subnormals)."""
+    zero: no NaN code (S.1111.111) ever appears, the scale is a finite positive
+    power of two, the value comes back within the E4M3 bound (half a step:
+    2^-4 relative for normals, 2^-10 * scale for subnormals), and the
+    dequantised value is exact in bf16 (except the top of the bf16 range,
+    where code x scale reaches 2^128)."""
     p = np.arange(1 << 16, dtype=np.uint32)
     p = p[((p >> 7) & 0xFF) != 0xFF].astype(np.uint16)
     x = np.zeros((len(p), 2), dtype=np.uint16)
@@ -119,10 +143,16 @@ def test_fp8_every_bf16_row_maximum_gives_finite_codes():
     codes, sc = quant.fp8_quantize_rows(x)
     assert not np.any((codes & 0x7F) == 0x7F)
     assert np.all(np.isfinite(sc)) and np.all(sc > 0)
+    assert np.all(np.frexp(sc.astype(np.float64))[0] == 0.5)
     xf = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    err = np.abs(quant.fp8_dequantize_rows(codes, sc) - xf)
+    deq = quant.fp8_dequantize_rows(codes, sc)
+    err = np.abs(deq - xf)
     bound = np.maximum(np.abs(xf) * 2.0 ** -4, sc[:, None].astype(np.float64) * 2.0 ** -10)
     assert np.all(err <= bound * (1 + 1e-6))
+    fin = np.abs(deq) < 2.0 ** 128
+    d32 = deq[fin].astype(np.float32)
+    assert np.all(d32.astype(np.float64) == deq[fin]) and np.all((d32.view(np.uint32) & 0xFFFF) == 0)
+    assert np.count_nonzero(~fin) <= 16
 
 
 def test_nvfp4_blocks_error_bound_and_packing():
