@@ -65,7 +65,10 @@ typedef struct ll_kv_cache ll_kv_cache;      /* opaque; owns the cache memory */
 
 typedef enum {
   LL_KV_BF16 = 0,       /* K/V stored as bf16 */
-  LL_KV_FP8_E4M3 = 1,   /* E4M3 codes + one fp32 scale per (token, head) row */
+  LL_KV_FP8_E4M3 = 1,   /* E4M3 codes + one fp32 scale per (token, head) row: the
+                           smallest power of two 2^k >= amax/448 with k >= -124
+                           (1 for an all-zero row); codes = E4M3(x / scale),
+                           round to nearest even, saturating */
   LL_KV_NVFP4 = 2       /* E2M1 codes, 16-value blocks along D, E4M3 block scale */
 } ll_kv_dtype;
 
@@ -190,8 +193,9 @@ LL_API ll_status ll_kv_recache_write(ll_kv_cache *cache, int layer, const void *
  *   of the same chunk. bf16 operands, fp32 accumulation and softmax, the
  *   probabilities rounded to bf16 for the PV product, bf16 output.
  *   Quantised caches: the layer's held frames are first dequantised into the
- *   cache's bf16 view (FP8: E4M3 x row scale rounded to bf16; NVFP4: E2M1 x
- *   E4M3 block scale, exact in bf16), then attended to like a bf16 cache. The
+ *   cache's bf16 view (FP8: E4M3 x power-of-two row scale; NVFP4: E2M1 x
+ *   E4M3 block scale; both exact in bf16), then attended to like a bf16
+ *   cache, so the attention sees exactly the dequantised values. The
  *   view is shared by all layers, so attention calls on one quantised cache
  *   must be ordered (one stream, or events).
  *   Pages: dpshk.com sec. 五/六; techwalker.com sec. 四/六; wmrh.cn sec. 6.  */

@@ -94,6 +94,19 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&x)[8]) {
   }
 }
 
+// log2 of the FP8 row scale: the smallest k >= -124 with amax <= 448 * 2^k
+// (0 for amax == 0). amax lies in [2^E, 2^(E+1)), so amax/448 lies in
+// (2^(E-9), 2^(E-7)) and k is E-8 or E-7: E-8 exactly when amax <= 448 * 2^(E-8)
+// = 1.75 * 2^E. Below 2^-118 the floor applies (amax/448 < 2^-126).
+__device__ __forceinline__ int fp8_scale_log2(float amax) {
+  if (amax == 0.f) return 0;
+  const int eb = static_cast<int>(__float_as_uint(amax) >> 23);   // biased exponent, amax >= 0
+  if (eb < 9) return -124;
+  const float thr = __uint_as_float((static_cast<uint32_t>(eb) << 23) | 0x600000u);   // 1.75 * 2^E
+  const int k = eb - 127 - 8 + (amax > thr ? 1 : 0);
+  return k < -124 ? -124 : k;
+}
+
 // Stores one 16-byte vector (8 values) of K and the same vector of V of one
 // (token, head) row at row `drow` of planes plane_k / plane_v, quantising for
 // FP8 (per-row scale) and NVFP4 (16-value blocks). The D/8 lanes of a row must
@@ -113,9 +126,9 @@ __device__ __forceinline__ void store_kv_vec(uint8_t *data, uint8_t *scales, lon
       *dv = vv;
     }
   } else if constexpr (FMT == FMT_FP8) {
-    // per (token, head) row: scale = max(amax/448, 2^-126) (1 if amax == 0),
-    // codes = E4M3(x * (1/scale)); the floor (smallest normal fp32) keeps 1/scale
-    // finite for rows whose maximum is below 448 * 2^-126
+    // per (token, head) row: scale = the smallest power of two 2^k with
+    // amax <= 448 * 2^k, k >= -124 (1 if amax == 0); codes = E4M3(x * 2^-k).
+    // Both the quotient and code x scale are then exact (the latter in bf16).
 #pragma unroll
     for (int kv = 0; kv < 2; ++kv) {
       float x[8];
@@ -124,8 +137,9 @@ __device__ __forceinline__ void store_kv_vec(uint8_t *data, uint8_t *scales, lon
 #pragma unroll
       for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
       for (int o = 1; o < vpr; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const float scale = amax == 0.f ? 1.0f : fmaxf(__fdiv_rn(amax, 448.0f), 0x1p-126f);
-      const float inv = __fdiv_rn(1.0f, scale);
+      const int k = fp8_scale_log2(amax);
+      const float scale = __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+      const float inv = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
       float y[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(x[e], inv);
@@ -138,7 +152,8 @@ __device__ __forceinline__ void store_kv_vec(uint8_t *data, uint8_t *scales, lon
       }
     }
   } else {
-    // NVFP4: per 16-value block (two lanes): sb = E4M3(amax/6); codes = E2M1(x / sb), 0 if sb == 0
+    // NVFP4: per 16-value block (two lanes): sb = E4M3(amax/6); codes = E2M1(x / sb)
+    // (IEEE division, then the hardware round-to-nearest-even), all +0 if sb == 0
 #pragma unroll
     for (int kv = 0; kv < 2; ++kv) {
       float x[8];
@@ -266,7 +281,9 @@ namespace llk {
 // once per attention call into the cache's bf16 view [2H][slots][D], which the
 // bf16 attention kernel then reads through TMA; every query tile of a head
 // shares the converted rows instead of converting them again.
-//   FP8:   e4m3 -> f16 (exact) -> fp32, times the row scale, to bf16 (nearest even)
+//   FP8:   e4m3 -> f16 (exact) -> fp32, times the row scale (a power of two at
+//          or above 2^-124): the product has at most 4 significant bits and
+//          lies at or above 2^-133, so it and its bf16 conversion are exact
 //   NVFP4: e2m1 -> f16 and E4M3 block scale -> f16 (both exact); the product has
 //          at most 6 significant bits and lies inside the f16 range, so it is
 //          exact, and so is its bf16 conversion.
