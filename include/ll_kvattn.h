@@ -216,6 +216,49 @@ LL_API ll_status ll_attn_sink_window_append(const void *q, const void *k_cur, co
  *   Synchronises the device first so that no enqueued work still uses it.  */
 LL_API ll_status ll_kv_cache_destroy(ll_kv_cache *cache);
 
+/* ---- sequence-parallel inference: the local steps around the exchange ---
+ * LongLive-2.0 explainer (wmrh.cn), sec. 18.3: inference can run sequence
+ * parallel across GPUs; sec. 15.2: a low-precision KV cache then also reduces
+ * the traffic between them. Head-sharded form used here: P ranks each hold
+ * N_s = N/P tokens of the chunk ([N_s][H][D] q, k_cur, v_cur) and a cache of
+ * H/P heads (rank r: heads r*H/P .. (r+1)*H/P-1). The caller's all-to-all
+ * (equal splits, e.g. NCCL) exchanges what ll_sp_pack_heads (or
+ * ll_sp_pack_heads_fp8) prepared; what rank r receives, [P][N_s][H/P][D] from
+ * ranks 0..P-1, is the whole chunk [N][H/P][D] for its heads: attention and
+ * append take it as is. The outputs [N][H/P][D] go back through a second
+ * all-to-all and ll_sp_unpack_heads. Heads never interact inside attention, so
+ * each rank's results are those of an unsharded cache for the same heads.
+ * Shared rules: head_dim 64 or 128; heads divisible by ranks (else
+ * LL_ERR_INVALID_ARG); device pointers, 16-byte aligned, caller-owned; work is
+ * only enqueued on `stream`; nothing is allocated.                          */
+
+/* [tokens][heads][D] bf16 -> [ranks][tokens][heads/ranks][D] bf16: the block
+ * for rank r holds heads r*heads/ranks.. of every token, contiguous. x and
+ * packed must not overlap.                                                   */
+LL_API ll_status ll_sp_pack_heads(const void *x, int tokens, int heads, int head_dim, int ranks, void *packed,
+                                  ll_stream_t stream);
+
+/* The inverse: [ranks][tokens][heads/ranks][D] -> [tokens][heads][D]. Used on
+ * the outputs after the return all-to-all (block r = heads of rank r).       */
+LL_API ll_status ll_sp_unpack_heads(const void *packed, int tokens, int heads, int head_dim, int ranks, void *x,
+                                    ll_stream_t stream);
+
+/* As ll_sp_pack_heads, but each (token, head) row is sent in the cache's FP8
+ * row format: codes [ranks][tokens][heads/ranks][D] E4M3 bytes and scales
+ * [ranks][tokens][heads/ranks] fp32, the scale the smallest power of two 2^k
+ * >= max|row|/448 (k >= -124; 1 for a zero row), codes round to nearest even,
+ * saturating - D + 4 bytes per row on the links instead of 2D. For K and V
+ * (sec. 15.2's quantised-KV communication); the receiver restores bf16 rows
+ * with ll_sp_dequant_fp8 before attention and append, which therefore see
+ * the FP8-rounded chunk.                                                     */
+LL_API ll_status ll_sp_pack_heads_fp8(const void *x, int tokens, int heads, int head_dim, int ranks, void *codes,
+                                      void *scales, ll_stream_t stream);
+
+/* FP8 rows [rows][D] codes + [rows] fp32 power-of-two scales -> [rows][D]
+ * bf16, code x scale (exact in bf16).                                        */
+LL_API ll_status ll_sp_dequant_fp8(const void *codes, const void *scales, long long rows, int head_dim, void *x,
+                                   ll_stream_t stream);
+
 /* ---- helpers --------------------------------------------------------- */
 
 /* Static string for a status code. Never NULL.                              */

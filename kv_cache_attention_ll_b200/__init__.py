@@ -42,6 +42,10 @@ _sig = {
     "ll_attn_sink_window_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _ll, _vp, _vp]),
     "ll_debug_wait_selftest": (_i, [_vp, _vp]),
     "ll_noalloc_debug_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i, _vp]),
+    "ll_sp_pack_heads": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
+    "ll_sp_unpack_heads": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
+    "ll_sp_pack_heads_fp8": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "ll_sp_dequant_fp8": (_i, [_vp, _vp, _ll, _i, _vp, _vp]),
     "ll_kv_cache_create_multishot": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
     "ll_kv_shot_begin": (_i, [_vp, _i, _i, _vp]),
     "ll_kv_cache_held": (_i, [_vp, _i, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
@@ -254,6 +258,30 @@ def ll_noalloc_debug_status(clear: bool = False, stream=None) -> int:
     if st not in (LL_OK, LL_ERR_TIMEOUT, LL_ERR_INVALID_ARG):
         _check(st, "ll_noalloc_debug_status")
     return w.value
+
+
+def ll_sp_pack_heads(x, tokens: int, heads: int, head_dim: int, ranks: int, packed, stream=None):
+    """[tokens][heads][D] -> [ranks][tokens][heads/ranks][D] (bf16)."""
+    _check(_lib.ll_sp_pack_heads(_ptr(x), tokens, heads, head_dim, ranks, _ptr(packed), _stream(stream)),
+           "ll_sp_pack_heads")
+
+
+def ll_sp_unpack_heads(packed, tokens: int, heads: int, head_dim: int, ranks: int, x, stream=None):
+    """[ranks][tokens][heads/ranks][D] -> [tokens][heads][D] (bf16)."""
+    _check(_lib.ll_sp_unpack_heads(_ptr(packed), tokens, heads, head_dim, ranks, _ptr(x), _stream(stream)),
+           "ll_sp_unpack_heads")
+
+
+def ll_sp_pack_heads_fp8(x, tokens: int, heads: int, head_dim: int, ranks: int, codes, scales, stream=None):
+    """As ll_sp_pack_heads, each row as E4M3 codes + an fp32 power-of-two scale."""
+    _check(_lib.ll_sp_pack_heads_fp8(_ptr(x), tokens, heads, head_dim, ranks, _raw_ptr(codes), _raw_ptr(scales),
+                                     _stream(stream)), "ll_sp_pack_heads_fp8")
+
+
+def ll_sp_dequant_fp8(codes, scales, rows: int, head_dim: int, x, stream=None):
+    """FP8 rows (codes, scales) -> bf16 rows [rows][D]."""
+    _check(_lib.ll_sp_dequant_fp8(_raw_ptr(codes), _raw_ptr(scales), rows, head_dim, _ptr(x), _stream(stream)),
+           "ll_sp_dequant_fp8")
 
 
 def _raw_ptr(x) -> int:

@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libll_kvattn.so")
-SOURCES = [os.path.join(HERE, "csrc", "ll_kvattn.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "ll_kvattn.cu"), os.path.join(HERE, "csrc", "sp_exchange.cu")]
 DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("attn_sink_window.cuh", "kv_scatter.cuh",
                                                            "sm100_ptx.cuh", "cache_layout.cuh")] + [
     os.path.join(ROOT, "include", "ll_kvattn.h")]
