@@ -338,12 +338,22 @@ LL_API ll_status ll_noalloc_debug_status(unsigned int *word, int clear, ll_strea
 
 /* Device-side status word of the cache's kernels: 0 = fine; otherwise OR-ed
  * flags, reasons in the low byte (1 = a bounded in-kernel wait gave up,
- * 2 = a recache addressed frames a layer does not hold) and the reporting
+ * 2 = a recache addressed frames a layer does not hold, 4 = an index check of
+ * the bounds-checking build failed) and the reporting
  * kernels in the next (1 = attention, 2 = append/recache, 4 = self-test).
  * Reading synchronises `stream`; `clear` resets it to 0. The call returns
  * LL_ERR_TIMEOUT if reason 1 is set, LL_ERR_INVALID_ARG for any other
  * non-zero word, LL_OK for 0; *word is filled in all three cases.          */
 LL_API ll_status ll_debug_status(ll_kv_cache *cache, unsigned int *word, int clear, ll_stream_t stream);
+
+/* Stray-write check: every region of a cache's allocation (data, scales,
+ * status word, counters, completion counts, view) is followed by a guard of
+ * canary bytes, filled at create and touched by nothing afterwards. This
+ * synchronises the cache's device, reads every guard back and returns LL_OK if
+ * all are intact; otherwise LL_ERR_INVALID_ARG, with *bad_offset (may be NULL)
+ * the allocation offset of the first changed byte. Not callable while
+ * capturing a stream.                                                        */
+LL_API ll_status ll_debug_check_canaries(const ll_kv_cache *cache, size_t *bad_offset);
 
 /* Self-test of the in-kernel failure path: launches one thread that waits, with
  * the kernels' bounded mbarrier wait, on a barrier that nothing ever completes.
@@ -351,6 +361,19 @@ LL_API ll_status ll_debug_status(ll_kv_cache *cache, unsigned int *word, int cle
  * cache's status word and returns; read it with ll_debug_status (expect
  * LL_ERR_TIMEOUT). The context stays usable. Faults nothing, hangs nothing.   */
 LL_API ll_status ll_debug_wait_selftest(ll_kv_cache *cache, ll_stream_t stream);
+
+/* Bounds-checking build. The library built with LL_BOUNDS_CHECK defined
+ * (libll_kvattn_debug.so) checks, before each access, the slot rows, planes
+ * and source vectors that the append/recache, dequantise and attention kernels
+ * compute, and every cache tile a TMA load addresses; an index outside its
+ * buffer sets reason 4 (with the kernel id) in the cache's status word and the
+ * access is skipped (a cache tile is replaced by row 0). Nothing traps or
+ * asserts. ll_bounds_checked() returns 1 in that build, 0 in the regular one.
+ * ll_debug_bounds_selftest runs one failing check on the cache's status word
+ * (kernel id 4, reason 4), in either build, to exercise the reporting path;
+ * nothing is accessed.                                                        */
+LL_API int ll_bounds_checked(void);
+LL_API ll_status ll_debug_bounds_selftest(ll_kv_cache *cache, ll_stream_t stream);
 
 /* Test hook: when the environment variable LL_KVATTN_TEST_FAIL_ALLOC is set to
  * a non-empty value other than "0", ll_kv_cache_create fails as if the device

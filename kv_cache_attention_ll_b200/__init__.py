@@ -7,7 +7,8 @@ Raw integer device pointers are accepted too.
 
 Importing this module loads the in-tree library and fails loudly if it is
 missing (build it with `python kv_cache_attention_ll_b200/build.py`); there is
-no fallback path.
+no fallback path. With LL_KVATTN_LIB=debug in the environment it loads the
+bounds-checking build instead (libll_kvattn_debug.so, built with --debug).
 """
 from __future__ import annotations
 
@@ -15,11 +16,14 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libll_kvattn.so")
+_VARIANT = os.environ.get("LL_KVATTN_LIB", "")
+if _VARIANT not in ("", "release", "debug"):
+    raise ImportError(f"LL_KVATTN_LIB={_VARIANT!r}: expected 'debug' or 'release'")
+LIB_PATH = os.path.join(_HERE, "libll_kvattn_debug.so" if _VARIANT == "debug" else "libll_kvattn.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build the CUDA library first "
-                      "(python kv_cache_attention_ll_b200/build.py); there is no fallback")
+                      "(python kv_cache_attention_ll_b200/build.py [--debug]); there is no fallback")
 _lib = ctypes.CDLL(LIB_PATH)
 
 LL_KV_BF16, LL_KV_FP8_E4M3, LL_KV_NVFP4 = 0, 1, 2
@@ -42,6 +46,9 @@ _sig = {
     "ll_attn_sink_window_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _ll, _vp, _vp]),
     "ll_debug_wait_selftest": (_i, [_vp, _vp]),
     "ll_noalloc_debug_status": (_i, [ctypes.POINTER(ctypes.c_uint), _i, _vp]),
+    "ll_debug_check_canaries": (_i, [_vp, ctypes.POINTER(_sz)]),
+    "ll_bounds_checked": (_i, []),
+    "ll_debug_bounds_selftest": (_i, [_vp, _vp]),
     "ll_sp_pack_heads": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
     "ll_sp_unpack_heads": (_i, [_vp, _i, _i, _i, _i, _vp, _vp]),
     "ll_sp_pack_heads_fp8": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp]),
@@ -291,6 +298,28 @@ def _raw_ptr(x) -> int:
     if not x.is_cuda or not x.is_contiguous():
         raise ValueError("buffers must be contiguous CUDA tensors")
     return x.data_ptr()
+
+
+def ll_debug_check_canaries(cache: KVCache) -> int:
+    """-1 if every guard byte around the cache's regions is intact, else the
+    allocation offset of the first changed byte."""
+    off = _sz()
+    st = _lib.ll_debug_check_canaries(cache.handle, ctypes.byref(off))
+    if st == LL_OK:
+        return -1
+    if st == LL_ERR_INVALID_ARG and off.value != ctypes.c_size_t(-1).value:
+        return off.value
+    _check(st, "ll_debug_check_canaries")
+    return -1
+
+
+def ll_bounds_checked() -> bool:
+    """True for the bounds-checking build of the library."""
+    return bool(_lib.ll_bounds_checked())
+
+
+def ll_debug_bounds_selftest(cache: KVCache, stream=None):
+    _check(_lib.ll_debug_bounds_selftest(cache.handle, _stream(stream)), "ll_debug_bounds_selftest")
 
 
 def ll_debug_wait_selftest(cache: KVCache, stream=None):

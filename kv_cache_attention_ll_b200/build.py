@@ -1,7 +1,9 @@
 """Build step of the CUDA library: compiles csrc/ into libll_kvattn.so for
-sm_100a, in-tree, next to this file. Run `python kv_cache_attention_ll_b200/build.py`
-or call build(); the Python binding loads the result and refuses to run
-without it."""
+sm_100a, in-tree, next to this file, and the bounds-checking build
+libll_kvattn_debug.so (LL_BOUNDS_CHECK: every computed slot, plane and tile
+index is checked before its access and a bad one is reported in the status
+word). Run `python kv_cache_attention_ll_b200/build.py [--debug]` or call
+build(); the Python binding loads the result and refuses to run without it."""
 from __future__ import annotations
 
 import os
@@ -11,9 +13,11 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libll_kvattn.so")
+LIB_DEBUG = os.path.join(HERE, "libll_kvattn_debug.so")
 SOURCES = [os.path.join(HERE, "csrc", "ll_kvattn.cu"), os.path.join(HERE, "csrc", "sp_exchange.cu")]
 DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("attn_sink_window.cuh", "kv_scatter.cuh",
                                                            "sm100_ptx.cuh", "cache_layout.cuh")] + [
+    os.path.abspath(__file__),
     os.path.join(ROOT, "include", "ll_kvattn.h")]
 
 
@@ -24,20 +28,20 @@ def nvcc_cmd(out: str = LIB, extra=()) -> list[str]:
             "-I", os.path.join(ROOT, "include"), "-o", out, *SOURCES, *extra]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(d) <= t for d in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if force or not up_to_date():
-        cmd = nvcc_cmd(extra=("-Xptxas", "-v") if verbose else ())
-        subprocess.run(cmd, check=True)
-    return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if force or not up_to_date(lib):
+        extra = (("-Xptxas", "-v") if verbose else ()) + (("-DLL_BOUNDS_CHECK",) if debug else ())
+        subprocess.run(nvcc_cmd(out=lib, extra=extra), check=True)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

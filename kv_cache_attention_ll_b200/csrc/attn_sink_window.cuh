@@ -72,6 +72,9 @@ struct AttnParams {
   int plane_v;           // (l*2 + 1) * H
   int num_q_tiles;
   float scale_log2;      // log2(e) / sqrt(D)
+  int map_rows;          // rows per plane and planes of tm_cache, and planes of the
+  int map_planes;        // cache itself (fused append): the bounds-checking build
+  int cache_planes;      // checks every tile coordinate and store against them
 };
 
 template <int D>
@@ -264,8 +267,15 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
       if (elect_one()) {
         mbar_arrive_expect_tx(k_full + st, C::TILE_BYTES);
         if (j < nc) {
+          int row0 = cache_tile_row(kr, j);
+          // (bounds-checking build) a tile outside the map is flagged and replaced
+          // by row 0, so that the barrier still completes
+          if (!LL_BOUNDS(row0 >= 0 && row0 + tile_valid(kr, j, prm.Tq) <= prm.map_rows &&
+                             prm.plane_v + h < prm.map_planes,
+                         prm.err, KID_ATTN))
+            row0 = 0;
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d(sk + b * C::BOX_BYTES, &prm.tm_cache, k_full + st, b * 64, cache_tile_row(kr, j), prm.plane_k + h);
+            tma_load_3d(sk + b * C::BOX_BYTES, &prm.tm_cache, k_full + st, b * 64, row0, prm.plane_k + h);
         } else {
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_3d(sk + b * C::BOX_BYTES, &prm.tm_kcur, k_full + st, b * 64, h, (j - nc) * C::BN);
@@ -277,8 +287,10 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
       if (elect_one()) {
         mbar_arrive_expect_tx(v_full + st, C::TILE_BYTES);
         if (j < nc) {
+          int row0 = cache_tile_row(kr, j);
+          if (!LL_BOUNDS(row0 >= 0 && row0 + tile_valid(kr, j, prm.Tq) <= prm.map_rows, prm.err, KID_ATTN)) row0 = 0;
           for (int b = 0; b < C::NBOX; ++b)
-            tma_load_3d(sv + b * C::BOX_BYTES, &prm.tm_cache, v_full + st, b * 64, cache_tile_row(kr, j), prm.plane_v + h);
+            tma_load_3d(sv + b * C::BOX_BYTES, &prm.tm_cache, v_full + st, b * 64, row0, prm.plane_v + h);
         } else {
           for (int b = 0; b < C::NBOX; ++b)
             tma_load_3d(sv + b * C::BOX_BYTES, &prm.tm_vcur, v_full + st, b * 64, h, (j - nc) * C::BN);
@@ -315,8 +327,8 @@ __global__ void __launch_bounds__(384, 1) attn_sink_window_kernel(const __grid_c
         const int t = q0 + r;                                  // token of the chunk
         const int fi = t / prm.T;
         const int slot = r < rows ? append_slot(p, shot_fill, ring_count, prm.G, prm.Ss, prm.R, prm.F, fi) : -1;
-        const bool act = slot >= 0;
         const long long drow = static_cast<long long>(slot) * prm.T + (t - fi * prm.T);
+        const bool act = slot >= 0 && LL_BOUNDS(drow < prm.slots && plane_v < prm.cache_planes, prm.err, KID_ATTN);
         uint4 vk = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
         if (act) {
           const long long src = (static_cast<long long>(t) * prm.H + h) * VPR + vec;

@@ -49,6 +49,8 @@ struct ScatterParams {
   unsigned *done;            // per-layer count of finished append blocks (zero between launches),
                              // kept away from the counters that every block reads
   unsigned *err;             // status word: recache beyond the held frames is flagged there
+  long long planes;          // planes of the cache (L*2*H), for the bounds-checking build
+  long long src_vec;         // 16-byte vectors of the source (all source layers and frames)
 };
 
 // 8 fp32 -> 8 E4M3 codes (round to nearest even, saturating), element 0 in byte 0
@@ -243,7 +245,9 @@ __global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) 
       nk = __ldg(q.src_k + src0 + i + stride);
       nv = __ldg(q.src_v + src0 + i + stride);
     }
-    store_kv_vec<FMT>(q.data, q.scales, plane_k, plane_v, q.slots, drow, q.D, vec, vk, vv, act);
+    const bool in = LL_BOUNDS(drow >= 0 && drow < q.slots && plane_v < q.planes && src0 + ic < q.src_vec, q.err,
+                              KID_SCATTER);
+    store_kv_vec<FMT>(q.data, q.scales, plane_k, plane_v, q.slots, drow, q.D, vec, vk, vv, act && in);
   }
   if (q.mode == SCATTER_APPEND) {
     // per layer, the last of its n_frames x gridDim.y blocks to finish advances
@@ -296,6 +300,8 @@ struct DequantParams {
   int H, D, slots, n_rows;
   int G, Ss, W, R, T;      // with ctr: the visible frame ranges of cache_layout.cuh are converted
   int plane0;              // first plane of the layer: layer * 2H
+  long long planes;        // planes of the codes and scales (bounds-checking build)
+  unsigned *err;           // status word (bounds-checking build), or null
 };
 
 __device__ __forceinline__ uint32_t f16x2_of_e4m3x2(uint32_t two_codes) {
@@ -342,6 +348,7 @@ __global__ void __launch_bounds__(256) kv_dequant_kernel(const DequantParams q) 
     const int vec = i % VPR;
     const int vr = i / VPR;                         // visible row
     const int row = vr < n0 ? r0 + vr : (vr < n0 + n1 ? r1 + (vr - n0) : r2 + (vr - n0 - n1));
+    if (!LL_BOUNDS(row >= 0 && row < q.slots && q.plane0 + lp < q.planes, q.err, KID_ATTN)) continue;
     const long long src_row = src_plane + row;
     uint32_t o[4];
     if constexpr (FMT == FMT_FP8) {

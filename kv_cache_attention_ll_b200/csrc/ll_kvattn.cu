@@ -46,11 +46,17 @@ struct ll_kv_cache {
   CUtensorMap tm_cache;       // bf16 cache planes (D, slots, L*2*H)
   uint8_t *view;              // quantised caches: bf16 view of one layer [2H][slots][D]
   CUtensorMap tm_view;        // (D, slots, 2H) over the view
+  std::vector<std::pair<size_t, size_t>> guards;  // canary ranges [begin, end) of the allocation
 };
 
 namespace {
 
 std::atomic<long long> g_alloc_count{0};
+
+// every region of a cache allocation is followed by a guard of this many extra
+// bytes (beyond the padding to 256), filled with kCanary at create
+constexpr size_t kGuardBytes = 256;
+constexpr int kCanary = 0xA5;
 
 bool test_fail_alloc() {
   const char *v = std::getenv("LL_KVATTN_TEST_FAIL_ALLOC");
@@ -196,6 +202,8 @@ ll_status launch_dequant(ll_kv_cache *c, int layer, cudaStream_t stream) {
   q.R = c->R;
   q.T = c->T;
   q.plane0 = layer * 2 * c->H;
+  q.planes = static_cast<long long>(c->L) * 2 * c->H;
+  q.err = c->err;
   return launch_dequant_kernel(q, c->dtype, c->device, stream);
 }
 
@@ -211,10 +219,12 @@ ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, int n_laye
   if (gy > 65535) gy = 65535;
   if (gy < 1) gy = 1;
   const dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(gy));
+  llk::ScatterParams p = q;
+  p.src_vec = pairs * q.frame_vec;
   switch (c->dtype) {
-    case LL_KV_BF16: llk::kv_scatter_kernel<llk::FMT_BF16><<<grid, 256, 0, stream>>>(q); break;
-    case LL_KV_FP8_E4M3: llk::kv_scatter_kernel<llk::FMT_FP8><<<grid, 256, 0, stream>>>(q); break;
-    case LL_KV_NVFP4: llk::kv_scatter_kernel<llk::FMT_NVFP4><<<grid, 256, 0, stream>>>(q); break;
+    case LL_KV_BF16: llk::kv_scatter_kernel<llk::FMT_BF16><<<grid, 256, 0, stream>>>(p); break;
+    case LL_KV_FP8_E4M3: llk::kv_scatter_kernel<llk::FMT_FP8><<<grid, 256, 0, stream>>>(p); break;
+    case LL_KV_NVFP4: llk::kv_scatter_kernel<llk::FMT_NVFP4><<<grid, 256, 0, stream>>>(p); break;
   }
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
@@ -239,6 +249,7 @@ llk::ScatterParams scatter_base(const ll_kv_cache *c, const void *k, const void 
   q.ctr = c->ctr;
   q.done = c->done;
   q.err = c->err;
+  q.planes = static_cast<long long>(c->L) * 2 * c->H;
   return q;
 }
 
@@ -320,18 +331,30 @@ ll_status create_cache(int layers, int heads, int head_dim, int tokens_per_frame
   const size_t data_plane = static_cast<size_t>(slots) * row_bytes;
   const size_t scale_plane = static_cast<size_t>(slots) * scale_row_bytes;
   const size_t data_bytes = data_plane * planes;
-  const size_t scale_off = (data_bytes + 255) & ~size_t(255);
   const size_t scale_bytes = scale_plane * planes;
-  const size_t err_off = (scale_off + scale_bytes + 255) & ~size_t(255);
-  // quantised caches also hold a bf16 view of one layer's K and V planes, the
-  // input of the attention kernel after each call's dequantisation
-  const size_t ctr_off = err_off + 256;
-  const size_t ctr_bytes = ((static_cast<size_t>(layers) * sizeof(llk::LayerCtr) + 255) / 256) * 256 +
-                           ((static_cast<size_t>(layers) * sizeof(unsigned) + 255) / 256) * 256;
-  const size_t view_off = ctr_off + ctr_bytes;
+  // Regions, each followed by a guard of canary bytes (the padding to the next
+  // 256-byte boundary plus kGuardBytes more): data | scales | status word |
+  // counters | append-completion counts | (quantised caches) the bf16 view of
+  // one layer's K and V planes, the input of the attention kernel after each
+  // call's dequantisation. ll_debug_check_canaries reads the guards back.
+  std::vector<std::pair<size_t, size_t>> guards;           // [begin, end) of each guard
+  size_t off = 0;
+  auto region = [&](size_t bytes) {
+    const size_t begin = off;
+    const size_t end = begin + bytes;
+    off = ((end + 255) & ~size_t(255)) + kGuardBytes;
+    guards.emplace_back(end, off);
+    return begin;
+  };
+  region(data_bytes);
+  const size_t scale_off = region(scale_bytes);
+  const size_t err_off = region(sizeof(unsigned));
+  const size_t ctr_off = region(static_cast<size_t>(layers) * sizeof(llk::LayerCtr));
+  const size_t done_off = region(static_cast<size_t>(layers) * sizeof(unsigned));
   const size_t view_bytes =
       kv_dtype == LL_KV_BF16 ? 0 : static_cast<size_t>(2 * heads) * slots * head_dim * 2;
-  const size_t total = view_off + view_bytes;
+  const size_t view_off = region(view_bytes);
+  const size_t total = off;
 
   if (test_fail_alloc()) return LL_ERR_OOM;
   int dev = 0;
@@ -360,10 +383,13 @@ ll_status create_cache(int layers, int heads, int head_dim, int tokens_per_frame
   c->scales = scale_bytes ? c->base + scale_off : nullptr;
   c->err = reinterpret_cast<unsigned *>(c->base + err_off);
   c->ctr = reinterpret_cast<llk::LayerCtr *>(c->base + ctr_off);
-  c->done = reinterpret_cast<unsigned *>(c->base + ctr_off +
-                                         ((static_cast<size_t>(layers) * sizeof(llk::LayerCtr) + 255) / 256) * 256);
+  c->done = reinterpret_cast<unsigned *>(c->base + done_off);
   c->view = view_bytes ? c->base + view_off : nullptr;
-  if (cudaMemset(mem, 0, total) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+  c->guards = guards;
+  bool filled = cudaMemset(mem, 0, total) == cudaSuccess;
+  for (const auto &g : guards)
+    filled = filled && cudaMemset(c->base + g.first, kCanary, g.second - g.first) == cudaSuccess;
+  if (!filled || cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(mem);
     g_alloc_count.fetch_sub(1);
     delete c;
@@ -438,6 +464,33 @@ ll_status ll_kv_cache_export(const ll_kv_cache *c, int layer, void *host_dst, si
       return LL_ERR_CUDA;
   }
   return cudaStreamSynchronize(s) == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+ll_status ll_debug_check_canaries(const ll_kv_cache *c, size_t *bad_offset) {
+  if (!c) return LL_ERR_INVALID_ARG;
+  if (bad_offset) *bad_offset = static_cast<size_t>(-1);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (cudaSetDevice(c->device) != cudaSuccess) return LL_ERR_CUDA;
+  ll_status r = cudaDeviceSynchronize() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+  std::vector<uint8_t> buf;
+  for (const auto &g : c->guards) {
+    if (r != LL_OK) break;
+    buf.resize(g.second - g.first);
+    if (cudaMemcpy(buf.data(), c->base + g.first, buf.size(), cudaMemcpyDeviceToHost) != cudaSuccess) {
+      r = LL_ERR_CUDA;
+      break;
+    }
+    for (size_t i = 0; i < buf.size(); ++i) {
+      if (buf[i] != static_cast<uint8_t>(kCanary)) {
+        if (bad_offset) *bad_offset = g.first + i;
+        r = LL_ERR_INVALID_ARG;
+        break;
+      }
+    }
+  }
+  cudaSetDevice(prev);
+  return r;
 }
 
 ll_status ll_debug_status(ll_kv_cache *c, unsigned int *word, int clear, ll_stream_t stream) {
@@ -554,6 +607,9 @@ ll_status attention(const void *q, const void *k_cur, const void *v_cur, ll_kv_c
   prm.plane_v = quantised ? c->H : (layer * 2 + 1) * c->H;
   prm.num_q_tiles = (Tq + 127) / 128;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(c->D)));
+  prm.map_rows = static_cast<int>(c->slots);
+  prm.cache_planes = c->L * 2 * c->H;
+  prm.map_planes = quantised ? 2 * c->H : prm.cache_planes;
   if (append) {
     prm.append = 1;
     prm.fmt = c->dtype == LL_KV_BF16 ? llk::FMT_BF16 : (c->dtype == LL_KV_FP8_E4M3 ? llk::FMT_FP8 : llk::FMT_NVFP4);
@@ -644,6 +700,29 @@ __global__ void wait_selftest_kernel(unsigned *err) {
   mbar_wait(&bar, 0, &abort_flag, err, KID_SELFTEST);
 }
 }  // namespace llk
+
+namespace llk {
+// The reporting path of the index checks: one check that fails; nothing is
+// accessed either way (the check decides only whether a store would happen).
+__global__ void bounds_selftest_kernel(unsigned *err) {
+  volatile int n = 1, idx = 1;
+  if (bounds_ok(idx < n, err, KID_SELFTEST)) atomicOr(err, 0u);
+}
+}  // namespace llk
+
+extern "C" ll_status ll_debug_bounds_selftest(ll_kv_cache *c, ll_stream_t stream) {
+  if (!c || !on_cache_device(c)) return LL_ERR_INVALID_ARG;
+  llk::bounds_selftest_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(c->err);
+  return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+extern "C" int ll_bounds_checked(void) {
+#ifdef LL_BOUNDS_CHECK
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 extern "C" ll_status ll_debug_wait_selftest(ll_kv_cache *c, ll_stream_t stream) {
   if (!c || !on_cache_device(c)) return LL_ERR_INVALID_ARG;
@@ -746,6 +825,8 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
     dq.R = window_frames;
     dq.T = tokens_per_frame;
     dq.plane0 = 0;
+    dq.planes = 2ll * heads;
+    dq.err = status;
     const ll_status ds = launch_dequant_kernel(dq, kv_dtype, dev, st);
     if (ds != LL_OK) return ds;
     long long tail_end = (static_cast<long long>(n_cache) + kKeyTile - 1) / kKeyTile * kKeyTile;
@@ -776,6 +857,9 @@ ll_status ll_attn_sink_window_noalloc(const void *q, const void *k_cur, const vo
   prm.plane_v = heads;
   prm.num_q_tiles = (Tq + 127) / 128;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(head_dim)));
+  prm.map_rows = static_cast<int>(slots);
+  prm.map_planes = 2 * heads;
+  prm.cache_planes = 2 * heads;
   const int grid = prm.num_q_tiles * heads;
   return head_dim == 128 ? launch_attn<128>(prm, grid, st) : launch_attn<64>(prm, grid, st);
 }

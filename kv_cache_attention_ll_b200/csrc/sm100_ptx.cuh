@@ -14,6 +14,7 @@ namespace llk {
 enum : unsigned {
   ERR_WAIT_TIMEOUT = 1u,     // a bounded wait gave up
   ERR_RANGE = 2u,            // a recache addressed frames the layer does not hold
+  ERR_BOUNDS = 4u,           // (bounds-checking build) an index fell outside its buffer; the access was skipped
   KID_ATTN = 1u << 8,
   KID_SCATTER = 2u << 8,
   KID_SELFTEST = 4u << 8,
@@ -23,6 +24,20 @@ enum : unsigned {
 // gives up: it records ERR_WAIT_TIMEOUT and reports failure to the caller, which
 // then winds the kernel down instead of spinning forever.
 constexpr long long kWaitLimitClocks = 1ll << 31;
+
+// Index checks of the bounds-checking build (compiled with LL_BOUNDS_CHECK):
+// LL_BOUNDS(cond, err, kid) is `cond`, and a false cond records ERR_BOUNDS and
+// the kernel id in the status word, so that the caller skips the access. In
+// the regular build it is `true` and costs nothing. Nothing traps or asserts.
+__device__ __forceinline__ bool bounds_ok(bool ok, unsigned *err, unsigned kid) {
+  if (!ok && err) atomicOr(err, kid | ERR_BOUNDS);
+  return ok;
+}
+#ifdef LL_BOUNDS_CHECK
+#define LL_BOUNDS(cond, err, kid) ::llk::bounds_ok((cond), (err), (kid))
+#else
+#define LL_BOUNDS(cond, err, kid) true
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -141,3 +141,14 @@ def test_header_is_plain_c_and_links(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert r.stdout.split() == ["in-kernel", "wait", "timed", "out", str(len(names))]
+
+
+def test_bounds_checking_build_loads_and_exports_every_symbol():
+    """The bounds-checking build is a second, complete copy of the library."""
+    import kv_cache_attention_ll_b200 as ll
+    path = os.path.join(os.path.dirname(ll.LIB_PATH), "libll_kvattn_debug.so")
+    lib = ctypes.CDLL(path)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    assert lib.ll_bounds_checked() == 1
+    assert ll.raw_lib().ll_bounds_checked() == 0

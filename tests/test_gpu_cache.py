@@ -70,6 +70,7 @@ def test_cache_bytes_match_oracle(kv_dtype, L, H, D, T, F, S, W):
                     pytest.fail(f"chunk {c} layer {l}: {len(bad)} bytes differ, first at {bad[0]} "
                                 f"(got {a[bad[0]]:#x}, want {b[bad[0]]:#x})")
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 
@@ -137,6 +138,7 @@ def test_constant_footprint_over_long_rollout():
         assert free1 == free0
         assert ll.ll_kv_cache_info(cache, 0)[0] == 320 * F
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 
@@ -187,5 +189,6 @@ def test_append_of_all_layers_in_one_launch(kv_dtype):
                 assert ll.ll_kv_cache_export(cache, l) == model.export(l), f"chunk {c} layer {l}"
                 assert ll.ll_kv_cache_info(cache, l)[0] == (c + 1) * F
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()

@@ -70,6 +70,7 @@ def test_fused_rollout_matches_oracle(kv_dtype, H, D, T, F, G, Ss, W, n, seed, m
             assert ll.ll_kv_cache_export(cache, 0) == model.export(0), f"cache bytes after chunk {c}"
             assert ll.ll_kv_cache_info(cache, 0)[0] == (c + 1) * F
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 
@@ -98,6 +99,7 @@ def test_fused_wan_shape_sampled_rows():
             model.append(0, k, v)
         assert ll.ll_kv_cache_export(cache, 0) == model.export(0)
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 

@@ -75,6 +75,7 @@ def test_multishot_rollout_matches_oracle(kv_dtype, H, D, T, F, G, Ss, W, n, see
             model.append(0, k, v)
             assert ll.ll_kv_cache_export(cache, 0) == model.export(0), f"cache bytes after chunk {c}"
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 
@@ -111,6 +112,7 @@ def test_multishot_recache_all_layers_bit_exact(kv_dtype):
         for l in range(L):
             assert ll.ll_kv_cache_export(cache, l) == model.export(l), f"layer {l}"
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 
@@ -147,6 +149,7 @@ def test_multishot_wan_shape_sampled_rows():
             model.append(0, k, v)
         assert ll.ll_kv_cache_export(cache, 0) == model.export(0)
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 

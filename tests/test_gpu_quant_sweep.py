@@ -159,6 +159,7 @@ def test_quantisers_bit_exact_on_crafted_rows(fmt):
         torch.cuda.synchronize()
         _assert_same(ll.ll_kv_cache_export(cache, 0), model.export(0), f"{fmt} recache")
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 
@@ -188,6 +189,7 @@ def test_fused_append_quantises_bit_exact_on_crafted_rows(fmt):
         torch.cuda.synchronize()
         _assert_same(ll.ll_kv_cache_export(cache, 0), model.export(0), f"{fmt} fused append")
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
 

@@ -7,7 +7,8 @@ window restart), recaches of random held ranges of one or all layers,
 attention and append (separate or fused) happen at random. After every
 operation the cache bytes of every layer must equal the oracle's cache model,
 and every attention output must match the fp64 oracle over the frames that the
-frame-classification definition names."""
+frame-classification definition names. At the end the canary bytes that guard
+every region of the cache allocation must be untouched (no stray writes)."""
 import random
 
 import numpy as np
@@ -89,5 +90,6 @@ def test_random_operation_sequence(seed):
                 assert ll.ll_kv_cache_export(cache, l) == model.export(l), f"seed {seed} chunk {c} layer {l}"
                 assert ll.ll_kv_cache_held(cache, l) == model.held3(l)
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()

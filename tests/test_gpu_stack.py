@@ -132,5 +132,6 @@ def test_wan_stack_with_prompt_switch():
             assert all(frame_src[ci[l]][f] is not None for f in _held(N_CHUNKS * F))
             assert ll.ll_kv_cache_export(cache, l) == model.export(ci[l]), f"layer {l} cache bytes"
         assert ll.ll_debug_status(cache) == 0
+        assert ll.ll_debug_check_canaries(cache) == -1, "a guard byte around the cache regions changed"
     finally:
         cache.close()
