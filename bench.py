@@ -727,9 +727,12 @@ def run_ours(args, world, rank, local):
         del ks_all, vs_all
 
     # ---- fused append: the same step with one launch per layer (attention and
-    # append together) on a cache with F spare ring slots
+    # append together) on a cache with F spare ring slots; off by default (it
+    # measured slower than the separate calls: the attention launch is bound
+    # by its softmax/MMA chain under the power cap, so the copy work inside it
+    # is not free, while the separate append runs at HBM speed)
     fused = None
-    if not args.no_fused:
+    if args.fused:
         fc = ll.ll_kv_cache_create_fused(L, H, D, T, F, S, 0, W)
         for c in range((S + W + F - 1) // F + 1):
             for l in range(L):
@@ -752,6 +755,46 @@ def run_ours(args, world, rank, local):
         fused = {"ms_per_step": f_ms, "value": world * ATTN_FLOP * L / (f_ms * 1e-3) / 1e12, "launches_per_step": L,
                  "cache_gb": ll.ll_kv_cache_info(fc, 0)[1] / 1e9, "device_status": ll.ll_debug_status(fc)}
         fc.close()
+
+    # ---- the local kernels of the head-sharded sequence-parallel step, one GPU:
+    # what one of P = 4 ranks runs around its two all-to-alls per layer, at the
+    # Wan shape (each rank holds 1170 tokens of the chunk for all 12 heads), over
+    # the 30 layers' inputs (larger than L2). HBM-bound permutations: bytes are
+    # what each kernel reads plus writes.
+    sp = None
+    if not args.no_sp:
+        P, ns = 4, TQ // 4
+        rows = ns * H
+        xs = [q[:ns].contiguous() for q in ks]
+        packed = [torch.empty_like(x) for x in xs]
+        codes = [torch.empty(rows * D, dtype=torch.uint8, device=dev) for _ in xs]
+        scl = [torch.empty(rows, dtype=torch.float32, device=dev) for _ in xs]
+        back = [torch.empty_like(x) for x in xs]
+        calls = {
+            "pack": (lambda l: ll.ll_sp_pack_heads(xs[l], ns, H, D, P, packed[l], stream), 2 * rows * D * 2),
+            "unpack": (lambda l: ll.ll_sp_unpack_heads(packed[l], ns, H, D, P, back[l], stream), 2 * rows * D * 2),
+            "pack_fp8": (lambda l: ll.ll_sp_pack_heads_fp8(xs[l], ns, H, D, P, codes[l], scl[l], stream),
+                         rows * D * 2 + rows * (D + 4)),
+            "dequant_fp8": (lambda l: ll.ll_sp_dequant_fp8(codes[l], scl[l], rows, D, back[l], stream),
+                            rows * (D + 4) + rows * D * 2),
+        }
+        sp = {"ranks": P, "tokens_per_rank": ns, "heads": H, "workload": "one rank of 4, Wan shape, 30 layers' inputs"}
+        for name, (fn, nbytes) in calls.items():
+            for l in range(L):
+                fn(l)
+            torch.cuda.synchronize(dev)
+            e0.record(stream)
+            for _ in range(3):
+                for l in range(L):
+                    fn(l)
+            e1.record(stream)
+            e1.synchronize()
+            us = e0.elapsed_time(e1) / (3 * L) * 1e3
+            sp[name] = {"us": us, "bytes": nbytes, "gbs": nbytes / (us * 1e-6) / 1e9,
+                        "frac_hbm": nbytes / (us * 1e-6) / 1e9 / peak_gbs}
+        n = TQ * (H // P) * D
+        sp["exchanged_bytes_per_rank_per_layer"] = {"plain": 8 * n, "fp8_kv": 4 * n + 2 * (n + 4 * TQ * (H // P))}
+        del xs, packed, codes, scl, back
 
     # ---- several shots (global sink + per-shot sink + window), same 12-frame
     # budget as the headline stack: global 3 + shot 3 + window 6. A shot starts
@@ -834,6 +877,7 @@ def run_ours(args, world, rank, local):
         "long_rollout": sweep,
         "multishot": multishot,
         "fused_append_step": fused,
+        "sp_exchange_kernels": sp,
         "batched_append_step": batched,
         "device_status": status,
     }
@@ -854,7 +898,9 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the window sweep / full-causal leg")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay leg")
     ap.add_argument("--no-multishot", action="store_true", help="skip the multi-shot cache leg")
-    ap.add_argument("--no-fused", action="store_true", help="skip the fused attention + append leg")
+    ap.add_argument("--no-fused", action="store_true", help="skip the batched-append leg")
+    ap.add_argument("--fused", action="store_true", help="also time the fused attention + append step")
+    ap.add_argument("--no-sp", action="store_true", help="skip the sequence-parallel exchange kernels leg")
     ap.add_argument("--no-library-context", action="store_true",
                     help="skip the cuDNN attention timing on the same problem")
     ap.add_argument("--layers", type=int, default=30, help="stack depth (30 = the Wan-1.3B stack)")
