@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libll_kvattn.so")
 LIB_DEBUG = os.path.join(HERE, "libll_kvattn_debug.so")
 SOURCES = [os.path.join(HERE, "csrc", "ll_kvattn.cu"), os.path.join(HERE, "csrc", "sp_exchange.cu")]
-DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("attn_sink_window.cuh", "kv_scatter.cuh",
+DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in ("attn_sink_window.cuh", "kv_scatter.cuh", "kv_codec.cuh",
                                                            "sm100_ptx.cuh", "cache_layout.cuh")] + [
     os.path.abspath(__file__),
     os.path.join(ROOT, "include", "ll_kvattn.h")]

@@ -39,7 +39,7 @@
 #include <cuda_bf16.h>
 
 #include "cache_layout.cuh"
-#include "kv_scatter.cuh"
+#include "kv_codec.cuh"
 #include "sm100_ptx.cuh"
 
 namespace llk {

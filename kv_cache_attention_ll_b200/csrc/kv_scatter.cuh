@@ -11,264 +11,320 @@
 //   recache (dpshk.com sec. 三.5; techwalker.com LONGLIVE article sec. 六): logical
 //            frame k of the held context (global sink, shot sink, window) to its
 //            slot (logical_slot)
-// Grid: blockIdx.x = one (source layer, source frame) pair, blockIdx.y strides
-// over that frame's T*H*D/8 16-byte vectors. Everything that depends on the
-// layer's frame counter (the destination slot, or that nothing is stored) is
-// decided once per block. One thread moves one vector (8 values) of K and the
-// same vector of V; the D/8 threads of one (token, head) row are consecutive
-// lanes, so reads are fully coalesced and each row is written as one
-// contiguous 128/256-byte run.
-// Quantising formats reduce the row (FP8) or the 16-value block (NVFP4) with
-// lane shuffles inside that group and write codes + scales.
+// Work split: the source rows ((token, head) pairs, D values each) are cut
+// into units of kRows rows of K and the same rows of V, 8 KB of bf16 each, and
+// every CTA owns a contiguous range of units. A producer warp copies whole
+// units into shared memory with cp.async.bulk (one instruction per 8 KB,
+// completion counted on the stage's mbarrier), so each CTA has kStages units in
+// flight from its first clocks; eight consumer warps take a stage, convert its
+// rows and store them to their planes, then hand the stage back. Everything
+// that depends on a layer's frame counters (the destination slot of a frame,
+// or that nothing is stored) is decided by the producer, once per unit.
+// A row is handled by D/16 consecutive lanes, 16 values each, so an FP8 row
+// maximum takes log2(D/16) shuffle rounds, an NVFP4 block is one lane's values,
+// and each row is written as one contiguous run of its plane.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cstdint>
 
 #include "cache_layout.cuh"
+#include "kv_codec.cuh"
 #include "sm100_ptx.cuh"
 
 namespace llk {
 
 enum ScatterMode : int { SCATTER_APPEND = 0, SCATTER_RECACHE = 1 };
-enum CacheFormat : int { FMT_BF16 = 0, FMT_FP8 = 1, FMT_NVFP4 = 2 };
 
 struct ScatterParams {
   const uint4 *src_k;        // [n_layers][n_frames*T][H][D] bf16
   const uint4 *src_v;
   uint8_t *data;             // cache data base (all layers)
   uint8_t *scales;           // cache scale base (quantised formats) or null
-  int frame_vec;             // T * H * (D/8): vectors of one frame (< 2^30)
-  int H, D, T, slots;        // slots = (S+W)*T per plane
+  int H, D, T, slots;        // slots = (G+Ss+R)*T rows per plane
   int layer0;                // first destination layer
+  int n_layers;              // source layers (consecutive destination layers)
   int n_frames;              // frames per source layer
   int mode;                  // ScatterMode
   int G, Ss, W, R, F;        // cache geometry: global sink, shot sink, window, ring slots, chunk frames
   int first;                 // recache: first logical frame
   LayerCtr *ctr;             // per-layer counters (device); append advances its layer's
-  unsigned *done;            // per-layer count of finished append blocks (zero between launches),
-                             // kept away from the counters that every block reads
-  unsigned *err;             // status word: recache beyond the held frames is flagged there
+  unsigned *done;            // per-layer count of append units whose counters were read (zero
+                             // between launches), kept away from the counters that CTAs read
+  unsigned *err;             // status word: recache beyond the held frames, a wait that gave up
   long long planes;          // planes of the cache (L*2*H), for the bounds-checking build
-  long long src_vec;         // 16-byte vectors of the source (all source layers and frames)
 };
 
-// 8 fp32 -> 8 E4M3 codes (round to nearest even, saturating), element 0 in byte 0
-__device__ __forceinline__ uint2 e4m3x8(const float (&y)[8]) {
-  uint32_t w[4];
+// Tile of the bulk scatter for head dimension D.
+template <int D>
+struct ScatterTile {
+  static constexpr int kLPR = D / 16;                   // lanes per row, 16 values each
+  static constexpr int kRows = 256 / kLPR;              // rows per unit: one pass of the 8 consumer warps
+  static constexpr int kRowBytes = D * 2;               // one bf16 source row
+  static constexpr int kUnitBytes = kRows * kRowBytes;  // 8 KB of K (and as much of V) per unit
+  static constexpr int kStages = 6;
+  static constexpr int kThreads = 288;                  // warps 0-7 consume, warp 8 produces
+  // stages, then per stage a full and an empty barrier (8 bytes each) and a
+  // unit record (16 bytes), then the abort flag
+  static constexpr int kBookBytes = kStages * (8 + 8 + 16) + 16;
+  static constexpr int kSmem = kStages * 2 * kUnitBytes + kBookBytes;
+  static_assert(kSmem <= 227 * 1024, "shared memory of one CTA");
+};
+
+// x / b from the correctly rounded reciprocal inv = 1/b: q = x * inv, the
+// residual r = x - q * b (exact, one fma), then q + r * inv rounded once
+// (Markstein's correction step), with the sign of x kept for x = -0. Away from
+// underflow this is the correctly rounded quotient; for the NVFP4 operands
+// (bf16 x, b an E4M3 value >= 2^-9 or 6) it can differ from it only where the
+// residual is subnormal (|x| < 2^-103, so |x / b| < 2^-94), where every E2M1
+// or E4M3 rounding gives zero.
+__device__ __forceinline__ float div_corrected(float x, float b, float inv) {
+  const float q = __fmul_rn(x, inv);
+  const float r = __fmaf_rn(-q, b, x);
+  return copysignf(__fmaf_rn(r, inv, q), x);
+}
+
+__device__ __forceinline__ float div_by_6(float x) {
+  constexpr float kInv6 = 1.0f / 6.0f;   // correctly rounded at compile time
+  return div_corrected(x, 6.0f, kInv6);
+}
+
+// E4M3 code of one fp32 value (round to nearest even, saturating)
+__device__ __forceinline__ uint32_t e4m3_code(float y) {
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(y));
+  return h & 0xFFu;
+}
+
+// One lane's 16 consecutive values (lo: the first 8, hi: the next 8) of row
+// `row` (= plane * slots + slot row) of a plane, quantised and stored (FP8 or
+// NVFP4). The kLPR lanes of a row are consecutive lanes and every lane of the
+// warp calls it: the FP8 row maximum is reduced with shuffles. Lanes with
+// act = false take part in the shuffles and store nothing.
+template <int FMT, int D>
+__device__ __forceinline__ void store_row16(uint8_t *data, uint8_t *scales, long long row, int j, const uint4 &lo,
+                                            const uint4 &hi, bool act) {
+  constexpr int kLPR = D / 16;
+  static_assert(FMT == FMT_FP8 || FMT == FMT_NVFP4, "quantised formats only");
+  {
+    float x0[8], x1[8];
+    bf16x8_to_f32(lo, x0);
+    bf16x8_to_f32(hi, x1);
+    float m0 = 0.f, m1 = 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint16_t h;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(y[2 * i + 1]), "f"(y[2 * i]));
-    w[i] = h;
-  }
-  return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-}
-
-// 8 fp32 -> 8 E2M1 codes packed in 4 bytes, element 2i in the low nibble of byte i
-__device__ __forceinline__ uint32_t e2m1x8(const float (&y)[8]) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(out)
-      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
-  return out;
-}
-
-// one E4M3 code -> its fp32 value (exact)
-__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
-  uint32_t h2;
-  // the code sits in both bytes, so either half of the f16 pair holds its value
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>((code & 0xFF) * 0x101u)));
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFF)));
-}
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float (&x)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
-// log2 of the FP8 row scale: the smallest k >= -124 with amax <= 448 * 2^k
-// (0 for amax == 0). amax lies in [2^E, 2^(E+1)), so amax/448 lies in
-// (2^(E-9), 2^(E-7)) and k is E-8 or E-7: E-8 exactly when amax <= 448 * 2^(E-8)
-// = 1.75 * 2^E. Below 2^-118 the floor applies (amax/448 < 2^-126).
-__device__ __forceinline__ int fp8_scale_log2(float amax) {
-  if (amax == 0.f) return 0;
-  const int eb = static_cast<int>(__float_as_uint(amax) >> 23);   // biased exponent, amax >= 0
-  if (eb < 9) return -124;
-  const float thr = __uint_as_float((static_cast<uint32_t>(eb) << 23) | 0x600000u);   // 1.75 * 2^E
-  const int k = eb - 127 - 8 + (amax > thr ? 1 : 0);
-  return k < -124 ? -124 : k;
-}
-
-// Stores one 16-byte vector (8 values) of K and the same vector of V of one
-// (token, head) row at row `drow` of planes plane_k / plane_v, quantising for
-// FP8 (per-row scale) and NVFP4 (16-value blocks). The D/8 lanes of a row must
-// be consecutive lanes of the warp, and every lane of the warp must call it:
-// the quantising formats reduce with shuffles. Lanes with act = false take
-// part in the shuffles and store nothing.
-template <int FMT>
-__device__ __forceinline__ void store_kv_vec(uint8_t *data, uint8_t *scales, long long plane_k, long long plane_v,
-                                             int slots, long long drow, int D, int vec, uint4 vk, uint4 vv,
-                                             bool act) {
-  const int vpr = D >> 3;
-  if constexpr (FMT == FMT_BF16) {
-    if (act) {
-      uint4 *dk = reinterpret_cast<uint4 *>(data) + (plane_k * slots + drow) * vpr + vec;
-      uint4 *dv = reinterpret_cast<uint4 *>(data) + (plane_v * slots + drow) * vpr + vec;
-      *dk = vk;
-      *dv = vv;
+    for (int e = 0; e < 8; ++e) {
+      m0 = fmaxf(m0, fabsf(x0[e]));
+      m1 = fmaxf(m1, fabsf(x1[e]));
     }
-  } else if constexpr (FMT == FMT_FP8) {
-    // per (token, head) row: scale = the smallest power of two 2^k with
-    // amax <= 448 * 2^k, k >= -124 (1 if amax == 0); codes = E4M3(x * 2^-k).
-    // Both the quotient and code x scale are then exact (the latter in bf16).
+    float amax = fmaxf(m0, m1);
+    if constexpr (FMT == FMT_FP8) {
+      // per (token, head) row: scale = the smallest power of two 2^k with
+      // amax <= 448 * 2^k, k >= -124 (1 if amax == 0); codes = E4M3(x * 2^-k)
 #pragma unroll
-    for (int kv = 0; kv < 2; ++kv) {
-      float x[8];
-      bf16x8_to_f32(kv == 0 ? vk : vv, x);
-      float amax = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
-      for (int o = 1; o < vpr; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      for (int o = 1; o < kLPR; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
       const int k = fp8_scale_log2(amax);
       const float scale = __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
       const float inv = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
-      float y[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(x[e], inv);
-      const uint2 codes = e4m3x8(y);
-      if (act) {
-        const long long plane = kv == 0 ? plane_k : plane_v;
-        uint2 *dc = reinterpret_cast<uint2 *>(data + (plane * slots + drow) * D) + vec;
-        *dc = codes;
-        if (vec == 0) reinterpret_cast<float *>(scales)[plane * slots + drow] = scale;
+      for (int e = 0; e < 8; ++e) {
+        x0[e] = __fmul_rn(x0[e], inv);
+        x1[e] = __fmul_rn(x1[e], inv);
       }
-    }
-  } else {
-    // NVFP4: per 16-value block (two lanes): sb = E4M3(amax/6); codes = E2M1(x / sb)
-    // (IEEE division, then the hardware round-to-nearest-even), all +0 if sb == 0
-#pragma unroll
-    for (int kv = 0; kv < 2; ++kv) {
-      float x[8];
-      bf16x8_to_f32(kv == 0 ? vk : vv, x);
-      float amax = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
-      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-      float sv[8] = {__fdiv_rn(amax, 6.0f), 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const uint32_t sb_code = e4m3x8(sv).x & 0xFFu;
-      const float sb = e4m3_to_f32(sb_code);
-      float y[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = sb == 0.f ? 0.f : __fdiv_rn(x[e], sb);
-      const uint32_t codes = sb == 0.f ? 0u : e2m1x8(y);
+      const uint2 c0 = e4m3x8(x0), c1 = e4m3x8(x1);
       if (act) {
-        const long long plane = kv == 0 ? plane_k : plane_v;
-        uint32_t *dc = reinterpret_cast<uint32_t *>(data + (plane * slots + drow) * (D / 2)) + vec;
-        *dc = codes;
-        if ((vec & 1) == 0) scales[(plane * slots + drow) * (D / 16) + (vec >> 1)] = static_cast<uint8_t>(sb_code);
+        *reinterpret_cast<uint4 *>(data + row * D + 16 * j) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+        if (j == 0) reinterpret_cast<float *>(scales)[row] = scale;
+      }
+    } else {
+      // NVFP4: the lane's 16 values are one block: sb = E4M3(amax/6);
+      // codes = E2M1(x / sb), round to nearest even, all +0 if sb == 0. Both
+      // quotients are a product with the correctly rounded reciprocal,
+      // corrected once with the exact residual (div_by_6 and below); the codes
+      // are those of the IEEE quotients for every bf16 input and E4M3 scale.
+      const uint32_t sb_code = e4m3_code(div_by_6(amax));
+      const float sb = e4m3_to_f32(sb_code);
+      uint32_t c0 = 0u, c1 = 0u;
+      if (sb != 0.f) {
+        const float inv = __frcp_rn(sb);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x0[e] = div_corrected(x0[e], sb, inv);
+          x1[e] = div_corrected(x1[e], sb, inv);
+        }
+        c0 = e2m1x8(x0);
+        c1 = e2m1x8(x1);
+      }
+      if (act) {
+        *reinterpret_cast<uint2 *>(data + row * (D / 2) + 8 * j) = make_uint2(c0, c1);
+        scales[row * (D / 16) + j] = static_cast<uint8_t>(sb_code);
       }
     }
   }
 }
 
-template <int FMT>
-__global__ void __launch_bounds__(256) kv_scatter_kernel(const ScatterParams q) {
-  const int vpr = q.D >> 3;                    // vectors per (token, head) row: 8 or 16
-  const int lg_vpr = vpr == 16 ? 4 : 3;
-  const int li = blockIdx.x / q.n_frames;      // source layer
-  const int fi = blockIdx.x % q.n_frames;      // source frame
-  const int layer = q.layer0 + li;
-  const long long src0 = static_cast<long long>(blockIdx.x) * q.frame_vec;   // first vector of the frame
-  const int stride = gridDim.y * blockDim.x;
-  // the source does not depend on the counters: each thread loads its first
-  // vectors now, while thread 0 reads the counters, and then stays one
-  // iteration ahead
-  uint4 nk = make_uint4(0, 0, 0, 0), nv = make_uint4(0, 0, 0, 0);
-  {
-    const int i0 = blockIdx.y * blockDim.x + threadIdx.x;
-    if (i0 < q.frame_vec) {
-      nk = __ldg(q.src_k + src0 + i0);
-      nv = __ldg(q.src_v + src0 + i0);
-    }
-  }
-  // the layer's counters, read once per block by thread 0 before the block's
-  // completion count below, so the append's advance (by the last block) comes
-  // after every block's read
-  __shared__ LayerCtr blk_ctr;
+template <int FMT, int D>
+__global__ void __launch_bounds__(ScatterTile<D>::kThreads, 2) kv_scatter_kernel(const ScatterParams q) {
+  using C = ScatterTile<D>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kStages * 2 * C::kUnitBytes);
+  uint64_t *empty = full + C::kStages;
+  int4 *unit_rec = reinterpret_cast<int4 *>(empty + C::kStages);   // (layer, slot or -1, first row, rows)
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(unit_rec + C::kStages);
+
+  const int rows_frame = q.T * q.H;                               // source rows of one frame
+  const int per_frame = (rows_frame + C::kRows - 1) / C::kRows;   // units of one frame
+  const long long per_layer = static_cast<long long>(q.n_frames) * per_frame;
+  const long long n_units = q.n_layers * per_layer;
+  const long long u0 = n_units * blockIdx.x / gridDim.x;
+  const long long u1 = n_units * (blockIdx.x + 1) / gridDim.x;
+  const int n_my = static_cast<int>(u1 - u0);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
   if (threadIdx.x == 0) {
-    const LayerCtr *lc = q.ctr + layer;
-    blk_ctr.p = __ldcg(&lc->p);
-    blk_ctr.ring_count = __ldcg(&lc->ring_count);
-    blk_ctr.ring_start = __ldcg(&lc->ring_start);
-    blk_ctr.shot_fill = __ldcg(&lc->shot_fill);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 8);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
   }
   __syncthreads();
-  const long long p = blk_ctr.p;
-  const long long ring_count = blk_ctr.ring_count;
-  const long long ring_start = blk_ctr.ring_start;
-  const int shot_fill = blk_ctr.shot_fill;
-  int slot;
-  if (q.mode == SCATTER_APPEND) {
-    slot = append_slot(p, shot_fill, ring_count, q.G, q.Ss, q.R, q.F, fi);
-  } else {
-    const HeldFrames hf = held_frames(p, shot_fill, ring_count, ring_start, q.G, q.W);
-    // recache of frames the layer does not hold: nothing of that layer is written
-    const bool reject = q.first + q.n_frames > hf.g + hf.sf + hf.w;
-    if (reject && fi == 0 && blockIdx.y == 0 && threadIdx.x == 0) atomicOr(q.err, KID_SCATTER | ERR_RANGE);
-    slot = reject ? -1 : logical_slot(hf, ring_count, q.G, q.Ss, q.R, q.first + fi);
-  }
-  // block-uniform trip count (slot is uniform too): every lane runs every
-  // iteration, so the row-group shuffles of the quantising formats see all 32
-  for (int base = slot < 0 ? q.frame_vec : blockIdx.y * blockDim.x; base < q.frame_vec; base += stride) {
-    const int i = base + threadIdx.x;
-    const bool act = i < q.frame_vec;
-    const int ic = act ? i : 0;
-    const int vec = ic & (vpr - 1);
-    const int row = ic >> lg_vpr;                           // token * H + head
-    const int t = row / q.H;
-    const int hh = row - t * q.H;
-    const long long plane_k = (static_cast<long long>(layer) * 2 + 0) * q.H + hh;
-    const long long plane_v = plane_k + q.H;
-    const long long drow = static_cast<long long>(slot) * q.T + t;   // row inside a plane
-    const uint4 vk = nk, vv = nv;                             // this iteration's vectors (loaded ahead)
-    if (i + stride < q.frame_vec) {
-      nk = __ldg(q.src_k + src0 + i + stride);
-      nv = __ldg(q.src_v + src0 + i + stride);
-    }
-    const bool in = LL_BOUNDS(drow >= 0 && drow < q.slots && plane_v < q.planes && src0 + ic < q.src_vec, q.err,
-                              KID_SCATTER);
-    store_kv_vec<FMT>(q.data, q.scales, plane_k, plane_v, q.slots, drow, q.D, vec, vk, vv, act && in);
-  }
-  if (q.mode == SCATTER_APPEND) {
-    // per layer, the last of its n_frames x gridDim.y blocks to finish advances
-    // the layer's counters; every block read them above, before its increment
-    // of the layer's completion count
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      __threadfence();
-      LayerCtr *c = q.ctr + layer;
-      const unsigned prev = atomicAdd(q.done + layer, 1u);
-      if (prev == static_cast<unsigned>(q.n_frames) * gridDim.y - 1) {
+
+  if (warp == 8) {
+    if (lane != 0) return;
+    // ---- producer: per unit, the slot of its frame (from the layer's
+    // counters, read when the CTA enters the layer), the unit record, the
+    // arrival with the byte count, and the two bulk copies ----
+    const char *src_k = reinterpret_cast<const char *>(q.src_k);
+    const char *src_v = reinterpret_cast<const char *>(q.src_v);
+    const long long src_rows = q.n_layers * static_cast<long long>(q.n_frames) * rows_frame;
+    (void)src_rows;                  // read by the bounds-checking build only
+    int issued = 0;                  // units handed to the consumers (in order)
+    int cur = -1, shot_fill = 0;
+    long long p = 0, ring_count = 0, ring_start = 0;
+    HeldFrames hf{0, 0, 0};
+    bool reject = false;
+    unsigned count_pending = 0;      // append: this CTA's units of layer `cur`, not yet counted
+    // The completion count of layer `cur` (append), taken when the CTA leaves
+    // the layer or has armed all its units: off the path of the copies and
+    // arrivals. The CTA whose count completes the layer advances its counters.
+    auto count_layer = [&]() {
+      if (!count_pending) return;
+      __threadfence();               // this CTA's counter read before its count
+      const unsigned prev = atomicAdd(q.done + cur, count_pending);
+      if (prev + count_pending == static_cast<unsigned>(per_layer)) {
         int fill;
         long long rc;
         append_advance(p, shot_fill, ring_count, q.G, q.Ss, q.F, &fill, &rc);
+        LayerCtr *c = q.ctr + cur;
         c->p = p + q.F;
         c->shot_fill = fill;
         c->ring_count = rc;
-        q.done[layer] = 0;
+        q.done[cur] = 0;
         __threadfence();
       }
+      count_pending = 0;
+    };
+    for (int jj = 0; jj < n_my; ++jj) {
+      const long long u = u0 + jj;
+      const int li = static_cast<int>(u / per_layer);
+      const int rem = static_cast<int>(u - li * per_layer);
+      const int fi = rem / per_frame;
+      const int row0 = (rem - fi * per_frame) * C::kRows;
+      const int nrows = rows_frame - row0 < C::kRows ? rows_frame - row0 : C::kRows;
+      const long long srow = (static_cast<long long>(li) * q.n_frames + fi) * rows_frame + row0;
+      const int layer = q.layer0 + li;
+      if (layer != cur) {
+        // the layer's counters, read once per CTA and layer before this CTA's
+        // completion count: the append's advance (by the CTA whose count
+        // completes the layer) comes after every CTA's read
+        count_layer();
+        cur = layer;
+        const LayerCtr *lc = q.ctr + layer;
+        p = __ldcg(&lc->p);
+        ring_count = __ldcg(&lc->ring_count);
+        ring_start = __ldcg(&lc->ring_start);
+        shot_fill = __ldcg(&lc->shot_fill);
+        if (q.mode == SCATTER_APPEND) {
+          const long long end = u1 < (li + 1) * per_layer ? u1 : (li + 1) * per_layer;
+          count_pending = static_cast<unsigned>(end - u);
+        } else {
+          hf = held_frames(p, shot_fill, ring_count, ring_start, q.G, q.W);
+          // recache of frames the layer does not hold: nothing of that layer is written
+          reject = q.first + q.n_frames > hf.g + hf.sf + hf.w;
+          if (reject && rem == 0) atomicOr(q.err, KID_SCATTER | ERR_RANGE);
+        }
+      }
+      if (*abort_flag) continue;     // keep the completion counts of the remaining layers
+      int slot;
+      if (q.mode == SCATTER_APPEND) slot = append_slot(p, shot_fill, ring_count, q.G, q.Ss, q.R, q.F, fi);
+      else slot = reject ? -1 : logical_slot(hf, ring_count, q.G, q.Ss, q.R, q.first + fi);
+      if (slot >= 0 && !LL_BOUNDS(srow >= 0 && srow + nrows <= src_rows, q.err, KID_SCATTER)) slot = -1;
+      const int s = jj % C::kStages;
+      if (jj >= C::kStages &&
+          !mbar_wait(&empty[s], ((jj / C::kStages) - 1) & 1, abort_flag, q.err, KID_SCATTER))
+        continue;
+      unit_rec[s] = make_int4(layer, slot, row0, nrows);
+      if (slot >= 0) {
+        const uint32_t bytes = static_cast<uint32_t>(nrows) * C::kRowBytes;
+        mbar_arrive_expect_tx(&full[s], 2 * bytes);
+        bulk_load(smem + (2 * s) * C::kUnitBytes, src_k + srow * C::kRowBytes, bytes, &full[s]);
+        bulk_load(smem + (2 * s + 1) * C::kUnitBytes, src_v + srow * C::kRowBytes, bytes, &full[s]);
+      } else {
+        mbar_arrive(&full[s]);       // nothing to copy: the consumers skip the unit
+      }
+      issued = jj + 1;
     }
+    count_layer();
+    // after an abort, copies may still be landing in this CTA's shared memory:
+    // wait (bounded) for the last phase issued on each stage before exiting
+    if (*abort_flag)
+      for (int jj = issued - C::kStages < 0 ? 0 : issued - C::kStages; jj < issued; ++jj)
+        mbar_wait_drain(&full[jj % C::kStages], (jj / C::kStages) & 1);
+    return;
+  }
+
+  // ---- consumers: warps 0-7, row r of each unit, 16 values per lane ----
+  const int r = threadIdx.x / C::kLPR;
+  const int j = threadIdx.x % C::kLPR;
+  // the two 16-byte halves of a lane's 32 bytes are read in an order that puts
+  // the 8 lanes of each quarter warp on 8 different bank groups
+  const int half_first = (threadIdx.x >> 2) & 1;
+  for (int jj = 0; jj < n_my; ++jj) {
+    const int s = jj % C::kStages;
+    if (!mbar_wait(&full[s], (jj / C::kStages) & 1, abort_flag, q.err, KID_SCATTER)) break;
+    const int4 rec = unit_rec[s];
+    if (rec.y >= 0) {
+      const int rf = rec.z + r;                  // row inside the frame: token * H + head
+      const int t = rf / q.H;
+      const int hh = rf - t * q.H;
+      const long long plane_k = static_cast<long long>(rec.x) * 2 * q.H + hh;
+      const long long drow = static_cast<long long>(rec.y) * q.T + t;
+      const bool act = r < rec.w &&
+                       LL_BOUNDS(drow < q.slots && plane_k + q.H < q.planes, q.err, KID_SCATTER);
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        const long long plane = plane_k + kv * q.H;
+        const uint8_t *srow = smem + (2 * s + kv) * C::kUnitBytes + r * C::kRowBytes;
+        if constexpr (FMT == FMT_BF16) {
+          const uint4 a = *reinterpret_cast<const uint4 *>(srow + 16 * j);
+          const uint4 c = *reinterpret_cast<const uint4 *>(srow + 16 * (j + C::kLPR));
+          if (act) {
+            uint4 *d = reinterpret_cast<uint4 *>(q.data + (plane * q.slots + drow) * D * 2);
+            d[j] = a;
+            d[j + C::kLPR] = c;
+          }
+        } else {
+          const uint8_t *src = srow + 32 * j;
+          const uint4 a = *reinterpret_cast<const uint4 *>(src + 16 * half_first);
+          const uint4 c = *reinterpret_cast<const uint4 *>(src + 16 * (1 - half_first));
+          store_row16<FMT, D>(q.data, q.scales, plane * q.slots + drow, j, half_first ? c : a, half_first ? a : c,
+                              act);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
   }
 }
 

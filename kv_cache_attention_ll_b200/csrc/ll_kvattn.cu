@@ -146,21 +146,24 @@ int num_sms(int device) {
   return n > 0 ? n : 148;
 }
 
+// Raises a kernel's dynamic shared-memory limit once per device (devices 0..63
+// remembered in `mask`; any other device sets it on every call).
+template <typename K>
+bool ensure_smem(K kernel, int bytes, std::atomic<unsigned long long> &mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+  if (bit && (mask.load() & bit)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  mask.fetch_or(bit);
+  return true;
+}
+
 template <int D>
 ll_status launch_attn(const llk::AttnParams &prm, int grid, cudaStream_t stream) {
   using C = llk::AttnCfg<D>;
-  // the shared-memory limit is raised once per device (devices 0..63 remembered;
-  // any other device sets it on every call)
-  static std::atomic<unsigned long long> configured_mask{0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
-  const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
-  if (!bit || !(configured_mask.load() & bit)) {
-    if (cudaFuncSetAttribute(llk::attn_sink_window_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_ALLOC) != cudaSuccess)
-      return LL_ERR_CUDA;
-    configured_mask.fetch_or(bit);
-  }
+  static std::atomic<unsigned long long> configured{0};
+  if (!ensure_smem(llk::attn_sink_window_kernel<D>, C::SMEM_ALLOC, configured)) return LL_ERR_CUDA;
   llk::attn_sink_window_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
@@ -207,26 +210,39 @@ ll_status launch_dequant(ll_kv_cache *c, int layer, cudaStream_t stream) {
   return launch_dequant_kernel(q, c->dtype, c->device, stream);
 }
 
-// Grid: one x-block per (source layer, source frame) pair, y-blocks striding
-// over the frame's vectors; about 8 blocks of 256 threads per SM in total.
-ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, int n_layers, cudaStream_t stream) {
-  const long long pairs = static_cast<long long>(n_layers) * q.n_frames;
-  if (pairs < 1 || pairs >= (1ll << 31)) return LL_ERR_INVALID_ARG;
-  const long long per_frame_blocks = (q.frame_vec + 255) / 256;
-  const long long target = static_cast<long long>(num_sms(c->device)) * 8;
-  long long gy = (target + pairs - 1) / pairs;
-  if (gy > per_frame_blocks) gy = per_frame_blocks;
-  if (gy > 65535) gy = 65535;
-  if (gy < 1) gy = 1;
-  const dim3 grid(static_cast<unsigned>(pairs), static_cast<unsigned>(gy));
-  llk::ScatterParams p = q;
-  p.src_vec = pairs * q.frame_vec;
-  switch (c->dtype) {
-    case LL_KV_BF16: llk::kv_scatter_kernel<llk::FMT_BF16><<<grid, 256, 0, stream>>>(p); break;
-    case LL_KV_FP8_E4M3: llk::kv_scatter_kernel<llk::FMT_FP8><<<grid, 256, 0, stream>>>(p); break;
-    case LL_KV_NVFP4: llk::kv_scatter_kernel<llk::FMT_NVFP4><<<grid, 256, 0, stream>>>(p); break;
-  }
+template <int FMT, int D>
+ll_status launch_scatter_kernel(const llk::ScatterParams &p, long long units, int device, cudaStream_t stream) {
+  using C = llk::ScatterTile<D>;
+  static std::atomic<unsigned long long> configured{0};
+  if (!ensure_smem(llk::kv_scatter_kernel<FMT, D>, C::kSmem, configured)) return LL_ERR_CUDA;
+  // two CTAs per SM, each owning a contiguous range of units (at least one)
+  long long grid = static_cast<long long>(num_sms(device)) * 2;
+  if (grid > units) grid = units;
+  llk::kv_scatter_kernel<FMT, D><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
+}
+
+// Units of D=128: 32 rows, D=64: 64 rows (8 KB of bf16 each, K and V apart).
+ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, int n_layers, cudaStream_t stream) {
+  const long long rows_frame = static_cast<long long>(q.T) * q.H;
+  const int unit_rows = 4096 / q.D;
+  const long long units = static_cast<long long>(n_layers) * q.n_frames * ((rows_frame + unit_rows - 1) / unit_rows);
+  if (units < 1 || units >= (1ll << 31)) return LL_ERR_INVALID_ARG;
+  llk::ScatterParams p = q;
+  p.n_layers = n_layers;
+  const int dev = c->device;
+  switch (c->dtype) {
+    case LL_KV_BF16:
+      return q.D == 128 ? launch_scatter_kernel<llk::FMT_BF16, 128>(p, units, dev, stream)
+                        : launch_scatter_kernel<llk::FMT_BF16, 64>(p, units, dev, stream);
+    case LL_KV_FP8_E4M3:
+      return q.D == 128 ? launch_scatter_kernel<llk::FMT_FP8, 128>(p, units, dev, stream)
+                        : launch_scatter_kernel<llk::FMT_FP8, 64>(p, units, dev, stream);
+    case LL_KV_NVFP4:
+      return q.D == 128 ? launch_scatter_kernel<llk::FMT_NVFP4, 128>(p, units, dev, stream)
+                        : launch_scatter_kernel<llk::FMT_NVFP4, 64>(p, units, dev, stream);
+  }
+  return LL_ERR_INVALID_ARG;
 }
 
 llk::ScatterParams scatter_base(const ll_kv_cache *c, const void *k, const void *v) {
@@ -239,7 +255,6 @@ llk::ScatterParams scatter_base(const ll_kv_cache *c, const void *k, const void 
   q.H = c->H;
   q.D = c->D;
   q.T = c->T;
-  q.frame_vec = c->T * c->H * (c->D / 8);
   q.slots = static_cast<int>(c->slots);
   q.G = c->S;
   q.Ss = c->Ss;

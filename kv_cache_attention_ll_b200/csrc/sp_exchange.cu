@@ -22,7 +22,7 @@
 #include <cstdint>
 
 #include "ll_kvattn.h"
-#include "kv_scatter.cuh"
+#include "kv_codec.cuh"
 
 namespace llk {
 
