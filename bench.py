@@ -52,8 +52,8 @@ def recache_bytes(layers: int) -> int:
 ATTN_MIN_BYTES = (4 * TQ + 2 * (S + W) * T) * H * D * 2   # q, k_cur, v_cur, out + cached K, V
 # ncu DRAM traffic of one attention launch at this shape and the hash of the
 # kernel sources it was taken with; reported only while the kernel is unchanged.
-ATTN_TRAFFIC = None            # re-captured after the sources changed
-ATTN_TRAFFIC_SRC_SHA = None
+ATTN_TRAFFIC = 165.0e6         # mean of the two captured launches (166.6 MB, 163.4 MB)
+ATTN_TRAFFIC_SRC_SHA = "0951aa36facdeeec"
 
 
 def _peaks():
@@ -483,6 +483,21 @@ def run_ours(args, world, rank, local):
         e1.synchronize()
         a_ms.append(e0.elapsed_time(e1) / L)
     app_ms = statistics.median(a_ms)
+    # a plain device copy of the same bytes (each layer's K and V), timed the
+    # same way: the size-matched scale for the append
+    ck, cv = torch.empty_like(ks[0]), torch.empty_like(vs[0])
+    c_ms = []
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.steps)):
+            e0.record(stream)
+            for l in range(L):
+                ck.copy_(ks[l])
+                cv.copy_(vs[l])
+            e1.record(stream)
+            e1.synchronize()
+            c_ms.append(e0.elapsed_time(e1) / L)
+    copy_ms = statistics.median(c_ms)
+    del ck, cv
 
     # ---- end to end through the C ABI from pinned host buffers
     def run_e2e():
@@ -596,11 +611,25 @@ def run_ours(args, world, rank, local):
                 qa.append(e0.elapsed_time(e1) / L)
             qa_ms = statistics.median(qa)
             qa_bytes = 2 * TQ * H * D * 2 + 2 * TQ * H * QUANT_ROW_BYTES[kvd]
+            # all-layer recache, quantising on write: reads the bf16 K/V of the
+            # held frames, writes codes and scales
+            qr = []
+            for _ in range(max(3, args.steps)):
+                e0.record(stream)
+                ll.ll_kv_recache_write(qc, -1, kn, vn, 0, S + W, stream)
+                e1.record(stream)
+                e1.synchronize()
+                qr.append(e0.elapsed_time(e1))
+            qr_ms = statistics.median(qr)
+            qr_bytes = 2 * L * (S + W) * T * H * (D * 2 + QUANT_ROW_BYTES[kvd])
             quant[kvd] = {"ms_per_step": q_ms, "value": ATTN_FLOP * L / (q_ms * 1e-3) / 1e12,
                           "attn_launch_ms": q_attn, "attn_tflops": ATTN_FLOP / (q_attn * 1e-3) / 1e12,
                           "append": {"ms_per_layer": qa_ms, "bytes": qa_bytes,
                                      "gbs": qa_bytes / (qa_ms * 1e-3) / 1e9,
                                      "frac_hbm": qa_bytes / (qa_ms * 1e-3) / 1e9 / peak_gbs},
+                          "recache": {"ms_all_layers": qr_ms, "bytes": qr_bytes,
+                                      "gbs": qr_bytes / (qr_ms * 1e-3) / 1e9,
+                                      "frac_hbm": qr_bytes / (qr_ms * 1e-3) / 1e9 / peak_gbs},
                           "cache_gb": qbytes / 1e9, "cache_gb_bf16": cache_bytes_bf16 / 1e9,
                           "device_status": ll.ll_debug_status(qc)}
             qc.close()
@@ -862,7 +891,8 @@ def run_ours(args, world, rank, local):
                      "kernel": "attn_sink_window_kernel<128>", "launch_ms": attn_avg,
                      "algorithmic_flop_per_launch": ATTN_FLOP, "min_bytes_per_launch": ATTN_MIN_BYTES},
         "append": {"ms_per_layer": app_ms, "gbs": APPEND_BYTES / (app_ms * 1e-3) / 1e9,
-                   "frac_hbm": APPEND_BYTES / (app_ms * 1e-3) / 1e9 / peak_gbs},
+                   "frac_hbm": APPEND_BYTES / (app_ms * 1e-3) / 1e9 / peak_gbs,
+                   "torch_copy_same_bytes_ms": copy_ms},
         "recache": {"ms_all_layers": rec_ms, "bytes": recache_bytes(L),
                     "gbs": recache_bytes(L) / (rec_ms * 1e-3) / 1e9,
                     "frac_hbm": recache_bytes(L) / (rec_ms * 1e-3) / 1e9 / peak_gbs},
