@@ -12,7 +12,7 @@
 //            frame k of the held context (global sink, shot sink, window) to its
 //            slot (logical_slot)
 // Work split: the source rows ((token, head) pairs, D values each) are cut
-// into units of kRows rows of K and the same rows of V, 8 KB of bf16 each, and
+// into units of kRows rows of K and the same rows of V (8 KB of bf16 each), and
 // every CTA owns a contiguous range of units. A producer warp copies whole
 // units into shared memory with cp.async.bulk (one instruction per 8 KB,
 // completion counted on the stage's mbarrier), so each CTA has kStages units in
@@ -55,14 +55,19 @@ struct ScatterParams {
   long long planes;          // planes of the cache (L*2*H), for the bounds-checking build
 };
 
-// Tile of the bulk scatter for head dimension D.
-template <int D>
+// Tile of the bulk scatter for head dimension D, with PASSES passes of the 8
+// consumer warps per unit: 8 KB units (6 stages) for the append, where the
+// launch is short and small units spread it over more CTAs, 16 KB units (3
+// stages) for the recache, a long stream where fewer, larger copies pay.
+template <int D, int PASSES>
 struct ScatterTile {
   static constexpr int kLPR = D / 16;                   // lanes per row, 16 values each
-  static constexpr int kRows = 256 / kLPR;              // rows per unit: one pass of the 8 consumer warps
+  static constexpr int kPasses = PASSES;
+  static constexpr int kPassRows = 256 / kLPR;          // rows of one pass
+  static constexpr int kRows = kPasses * kPassRows;     // rows per unit
   static constexpr int kRowBytes = D * 2;               // one bf16 source row
-  static constexpr int kUnitBytes = kRows * kRowBytes;  // 8 KB of K (and as much of V) per unit
-  static constexpr int kStages = 6;
+  static constexpr int kUnitBytes = kRows * kRowBytes;  // kPasses x 8 KB of K (and as much of V)
+  static constexpr int kStages = 6 / kPasses;
   static constexpr int kThreads = 288;                  // warps 0-7 consume, warp 8 produces
   // stages, then per stage a full and an empty barrier (8 bytes each) and a
   // unit record (16 bytes), then the abort flag
@@ -162,9 +167,9 @@ __device__ __forceinline__ void store_row16(uint8_t *data, uint8_t *scales, long
   }
 }
 
-template <int FMT, int D>
-__global__ void __launch_bounds__(ScatterTile<D>::kThreads, 2) kv_scatter_kernel(const ScatterParams q) {
-  using C = ScatterTile<D>;
+template <int FMT, int D, int PASSES>
+__global__ void __launch_bounds__(ScatterTile<D, PASSES>::kThreads, 2) kv_scatter_kernel(const ScatterParams q) {
+  using C = ScatterTile<D, PASSES>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kStages * 2 * C::kUnitBytes);
   uint64_t *empty = full + C::kStages;
@@ -284,8 +289,8 @@ __global__ void __launch_bounds__(ScatterTile<D>::kThreads, 2) kv_scatter_kernel
     return;
   }
 
-  // ---- consumers: warps 0-7, row r of each unit, 16 values per lane ----
-  const int r = threadIdx.x / C::kLPR;
+  // ---- consumers: warps 0-7, rows r0 + kPassRows * pass of each unit, 16 values per lane ----
+  const int r0 = threadIdx.x / C::kLPR;
   const int j = threadIdx.x % C::kLPR;
   // the two 16-byte halves of a lane's 32 bytes are read in an order that puts
   // the 8 lanes of each quarter warp on 8 different bank groups
@@ -294,7 +299,10 @@ __global__ void __launch_bounds__(ScatterTile<D>::kThreads, 2) kv_scatter_kernel
     const int s = jj % C::kStages;
     if (!mbar_wait(&full[s], (jj / C::kStages) & 1, abort_flag, q.err, KID_SCATTER)) break;
     const int4 rec = unit_rec[s];
-    if (rec.y >= 0) {
+#pragma unroll
+    for (int pass = 0; pass < C::kPasses; ++pass) {
+      if (rec.y < 0) break;
+      const int r = r0 + pass * C::kPassRows;
       const int rf = rec.z + r;                  // row inside the frame: token * H + head
       const int t = rf / q.H;
       const int hh = rf - t * q.H;

@@ -160,10 +160,21 @@ bool ensure_smem(K kernel, int bytes, std::atomic<unsigned long long> &mask) {
 }
 
 template <int D>
+bool prepare_attn() {
+  static std::atomic<unsigned long long> configured{0};
+  return ensure_smem(llk::attn_sink_window_kernel<D>, llk::AttnCfg<D>::SMEM_ALLOC, configured);
+}
+
+template <int FMT, int D, int PASSES>
+bool prepare_scatter() {
+  static std::atomic<unsigned long long> configured{0};
+  return ensure_smem(llk::kv_scatter_kernel<FMT, D, PASSES>, llk::ScatterTile<D, PASSES>::kSmem, configured);
+}
+
+template <int D>
 ll_status launch_attn(const llk::AttnParams &prm, int grid, cudaStream_t stream) {
   using C = llk::AttnCfg<D>;
-  static std::atomic<unsigned long long> configured{0};
-  if (!ensure_smem(llk::attn_sink_window_kernel<D>, C::SMEM_ALLOC, configured)) return LL_ERR_CUDA;
+  if (!prepare_attn<D>()) return LL_ERR_CUDA;
   llk::attn_sink_window_kernel<D><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(prm);
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
@@ -210,37 +221,41 @@ ll_status launch_dequant(ll_kv_cache *c, int layer, cudaStream_t stream) {
   return launch_dequant_kernel(q, c->dtype, c->device, stream);
 }
 
-template <int FMT, int D>
-ll_status launch_scatter_kernel(const llk::ScatterParams &p, long long units, int device, cudaStream_t stream) {
-  using C = llk::ScatterTile<D>;
-  static std::atomic<unsigned long long> configured{0};
-  if (!ensure_smem(llk::kv_scatter_kernel<FMT, D>, C::kSmem, configured)) return LL_ERR_CUDA;
+template <int FMT, int D, int PASSES>
+ll_status launch_scatter_kernel(const llk::ScatterParams &p, int device, cudaStream_t stream) {
+  using C = llk::ScatterTile<D, PASSES>;
+  const long long rows_frame = static_cast<long long>(p.T) * p.H;
+  const long long units = static_cast<long long>(p.n_layers) * p.n_frames * ((rows_frame + C::kRows - 1) / C::kRows);
+  if (units < 1 || units >= (1ll << 31)) return LL_ERR_INVALID_ARG;
+  if (!prepare_scatter<FMT, D, PASSES>()) return LL_ERR_CUDA;
   // two CTAs per SM, each owning a contiguous range of units (at least one)
   long long grid = static_cast<long long>(num_sms(device)) * 2;
   if (grid > units) grid = units;
-  llk::kv_scatter_kernel<FMT, D><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, stream>>>(p);
+  llk::kv_scatter_kernel<FMT, D, PASSES><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
 }
 
-// Units of D=128: 32 rows, D=64: 64 rows (8 KB of bf16 each, K and V apart).
+template <int FMT, int D>
+ll_status launch_scatter_mode(const llk::ScatterParams &p, int device, cudaStream_t stream) {
+  return p.mode == llk::SCATTER_APPEND ? launch_scatter_kernel<FMT, D, 1>(p, device, stream)
+                                       : launch_scatter_kernel<FMT, D, 2>(p, device, stream);
+}
+
+// Units of ScatterTile<D, passes>::kRows source rows, K and V apart.
 ll_status launch_scatter(ll_kv_cache *c, const llk::ScatterParams &q, int n_layers, cudaStream_t stream) {
-  const long long rows_frame = static_cast<long long>(q.T) * q.H;
-  const int unit_rows = 4096 / q.D;
-  const long long units = static_cast<long long>(n_layers) * q.n_frames * ((rows_frame + unit_rows - 1) / unit_rows);
-  if (units < 1 || units >= (1ll << 31)) return LL_ERR_INVALID_ARG;
   llk::ScatterParams p = q;
   p.n_layers = n_layers;
   const int dev = c->device;
   switch (c->dtype) {
     case LL_KV_BF16:
-      return q.D == 128 ? launch_scatter_kernel<llk::FMT_BF16, 128>(p, units, dev, stream)
-                        : launch_scatter_kernel<llk::FMT_BF16, 64>(p, units, dev, stream);
+      return q.D == 128 ? launch_scatter_mode<llk::FMT_BF16, 128>(p, dev, stream)
+                        : launch_scatter_mode<llk::FMT_BF16, 64>(p, dev, stream);
     case LL_KV_FP8_E4M3:
-      return q.D == 128 ? launch_scatter_kernel<llk::FMT_FP8, 128>(p, units, dev, stream)
-                        : launch_scatter_kernel<llk::FMT_FP8, 64>(p, units, dev, stream);
+      return q.D == 128 ? launch_scatter_mode<llk::FMT_FP8, 128>(p, dev, stream)
+                        : launch_scatter_mode<llk::FMT_FP8, 64>(p, dev, stream);
     case LL_KV_NVFP4:
-      return q.D == 128 ? launch_scatter_kernel<llk::FMT_NVFP4, 128>(p, units, dev, stream)
-                        : launch_scatter_kernel<llk::FMT_NVFP4, 64>(p, units, dev, stream);
+      return q.D == 128 ? launch_scatter_mode<llk::FMT_NVFP4, 128>(p, dev, stream)
+                        : launch_scatter_mode<llk::FMT_NVFP4, 64>(p, dev, stream);
   }
   return LL_ERR_INVALID_ARG;
 }
@@ -316,7 +331,48 @@ ll_status ll_kv_cache_create_fused(int layers, int heads, int head_dim, int toke
 
 }  // extern "C"
 
+namespace llk {
+// the shot start of ll_kv_shot_begin: empties the shot sink of layers
+// [l0, l0 + nl) and, if asked, restarts their window
+__global__ void shot_begin_kernel(LayerCtr *ctr, int l0, int nl, int clear_window) {
+  for (int i = threadIdx.x; i < nl; i += blockDim.x) {
+    LayerCtr *c = ctr + l0 + i;
+    c->shot_fill = 0;
+    if (clear_window) c->ring_start = c->ring_count;
+  }
+}
+}  // namespace llk
+
 namespace {
+// Loads every kernel a chunk step can launch (and raises the shared-memory
+// limits) once per device, at the first cache creation there: with lazy module
+// loading a kernel's first launch would otherwise take device memory for its
+// code in the middle of a rollout, after the cache's footprint is fixed.
+bool preload_kernels(int dev) {
+  static std::atomic<unsigned long long> loaded{0};
+  const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+  if (bit && (loaded.load() & bit)) return true;
+  bool ok = prepare_attn<64>() && prepare_attn<128>();
+  ok = ok && prepare_scatter<llk::FMT_BF16, 64, 1>() && prepare_scatter<llk::FMT_BF16, 64, 2>() &&
+       prepare_scatter<llk::FMT_BF16, 128, 1>() && prepare_scatter<llk::FMT_BF16, 128, 2>() &&
+       prepare_scatter<llk::FMT_FP8, 64, 1>() && prepare_scatter<llk::FMT_FP8, 64, 2>() &&
+       prepare_scatter<llk::FMT_FP8, 128, 1>() && prepare_scatter<llk::FMT_FP8, 128, 2>() &&
+       prepare_scatter<llk::FMT_NVFP4, 64, 1>() && prepare_scatter<llk::FMT_NVFP4, 64, 2>() &&
+       prepare_scatter<llk::FMT_NVFP4, 128, 1>() && prepare_scatter<llk::FMT_NVFP4, 128, 2>();
+  cudaFuncAttributes a;
+  ok = ok && cudaFuncGetAttributes(&a, llk::kv_dequant_kernel<llk::FMT_FP8, 8>) == cudaSuccess &&
+       cudaFuncGetAttributes(&a, llk::kv_dequant_kernel<llk::FMT_FP8, 16>) == cudaSuccess &&
+       cudaFuncGetAttributes(&a, llk::kv_dequant_kernel<llk::FMT_NVFP4, 8>) == cudaSuccess &&
+       cudaFuncGetAttributes(&a, llk::kv_dequant_kernel<llk::FMT_NVFP4, 16>) == cudaSuccess &&
+       cudaFuncGetAttributes(&a, llk::shot_begin_kernel) == cudaSuccess;
+  if (!ok) {
+    cudaGetLastError();
+    return false;
+  }
+  loaded.fetch_or(bit);
+  return true;
+}
+
 ll_status create_cache(int layers, int heads, int head_dim, int tokens_per_frame, int frames_per_chunk,
                        int global_sink_frames, int shot_sink_frames, int window_frames, bool spare_slots,
                        ll_kv_dtype kv_dtype, ll_kv_cache **out) {
@@ -374,6 +430,7 @@ ll_status create_cache(int layers, int heads, int head_dim, int tokens_per_frame
   if (test_fail_alloc()) return LL_ERR_OOM;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return LL_ERR_CUDA;
+  if (!preload_kernels(dev)) return LL_ERR_CUDA;
   ll_kv_cache *c = new (std::nothrow) ll_kv_cache();
   if (!c) return LL_ERR_OOM;
   c->L = layers; c->H = heads; c->D = head_dim; c->T = tokens_per_frame; c->F = frames_per_chunk;
@@ -652,18 +709,10 @@ ll_status attention(const void *q, const void *k_cur, const void *v_cur, ll_kv_c
 extern "C" {
 
 // ---------------------------------------------------------------------------
-// Shot start (several shots per video): empties the shot sink of the addressed
+// Shot start (several shots per video): shot_begin_kernel (above, before the
+// cache creation that preloads it) empties the shot sink of the addressed
 // layers and, if asked, restarts their window. A kernel, so that it is ordered
 // with the appends on the stream and can be recorded in a graph.
-namespace llk {
-__global__ void shot_begin_kernel(LayerCtr *ctr, int l0, int nl, int clear_window) {
-  for (int i = threadIdx.x; i < nl; i += blockDim.x) {
-    LayerCtr *c = ctr + l0 + i;
-    c->shot_fill = 0;
-    if (clear_window) c->ring_start = c->ring_count;
-  }
-}
-}  // namespace llk
 
 extern "C" ll_status ll_kv_shot_begin(ll_kv_cache *c, int layer, int clear_window, ll_stream_t stream) {
   if (!c || layer < -1 || layer >= c->L) return LL_ERR_INVALID_ARG;
