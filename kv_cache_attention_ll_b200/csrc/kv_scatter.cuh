@@ -111,58 +111,56 @@ __device__ __forceinline__ void store_row16(uint8_t *data, uint8_t *scales, long
                                             const uint4 &hi, bool act) {
   constexpr int kLPR = D / 16;
   static_assert(FMT == FMT_FP8 || FMT == FMT_NVFP4, "quantised formats only");
-  {
-    float x0[8], x1[8];
-    bf16x8_to_f32(lo, x0);
-    bf16x8_to_f32(hi, x1);
-    float m0 = 0.f, m1 = 0.f;
+  float x0[8], x1[8];
+  bf16x8_to_f32(lo, x0);
+  bf16x8_to_f32(hi, x1);
+  float m0 = 0.f, m1 = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    m0 = fmaxf(m0, fabsf(x0[e]));
+    m1 = fmaxf(m1, fabsf(x1[e]));
+  }
+  float amax = fmaxf(m0, m1);
+  if constexpr (FMT == FMT_FP8) {
+    // per (token, head) row: scale = the smallest power of two 2^k with
+    // amax <= 448 * 2^k, k >= -124 (1 if amax == 0); codes = E4M3(x * 2^-k)
+#pragma unroll
+    for (int o = 1; o < kLPR; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const int k = fp8_scale_log2(amax);
+    const float scale = __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
+    const float inv = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      m0 = fmaxf(m0, fabsf(x0[e]));
-      m1 = fmaxf(m1, fabsf(x1[e]));
+      x0[e] = __fmul_rn(x0[e], inv);
+      x1[e] = __fmul_rn(x1[e], inv);
     }
-    float amax = fmaxf(m0, m1);
-    if constexpr (FMT == FMT_FP8) {
-      // per (token, head) row: scale = the smallest power of two 2^k with
-      // amax <= 448 * 2^k, k >= -124 (1 if amax == 0); codes = E4M3(x * 2^-k)
-#pragma unroll
-      for (int o = 1; o < kLPR; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const int k = fp8_scale_log2(amax);
-      const float scale = __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
-      const float inv = __uint_as_float(static_cast<uint32_t>(127 - k) << 23);
+    const uint2 c0 = e4m3x8(x0), c1 = e4m3x8(x1);
+    if (act) {
+      *reinterpret_cast<uint4 *>(data + row * D + 16 * j) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+      if (j == 0) reinterpret_cast<float *>(scales)[row] = scale;
+    }
+  } else {
+    // NVFP4: the lane's 16 values are one block: sb = E4M3(amax/6);
+    // codes = E2M1(x / sb), round to nearest even, all +0 if sb == 0. Both
+    // quotients are a product with the correctly rounded reciprocal,
+    // corrected once with the exact residual (div_by_6 and below); the codes
+    // are those of the IEEE quotients for every bf16 input and E4M3 scale.
+    const uint32_t sb_code = e4m3_code(div_by_6(amax));
+    const float sb = e4m3_to_f32(sb_code);
+    uint32_t c0 = 0u, c1 = 0u;
+    if (sb != 0.f) {
+      const float inv = __frcp_rn(sb);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        x0[e] = __fmul_rn(x0[e], inv);
-        x1[e] = __fmul_rn(x1[e], inv);
+        x0[e] = div_corrected(x0[e], sb, inv);
+        x1[e] = div_corrected(x1[e], sb, inv);
       }
-      const uint2 c0 = e4m3x8(x0), c1 = e4m3x8(x1);
-      if (act) {
-        *reinterpret_cast<uint4 *>(data + row * D + 16 * j) = make_uint4(c0.x, c0.y, c1.x, c1.y);
-        if (j == 0) reinterpret_cast<float *>(scales)[row] = scale;
-      }
-    } else {
-      // NVFP4: the lane's 16 values are one block: sb = E4M3(amax/6);
-      // codes = E2M1(x / sb), round to nearest even, all +0 if sb == 0. Both
-      // quotients are a product with the correctly rounded reciprocal,
-      // corrected once with the exact residual (div_by_6 and below); the codes
-      // are those of the IEEE quotients for every bf16 input and E4M3 scale.
-      const uint32_t sb_code = e4m3_code(div_by_6(amax));
-      const float sb = e4m3_to_f32(sb_code);
-      uint32_t c0 = 0u, c1 = 0u;
-      if (sb != 0.f) {
-        const float inv = __frcp_rn(sb);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x0[e] = div_corrected(x0[e], sb, inv);
-          x1[e] = div_corrected(x1[e], sb, inv);
-        }
-        c0 = e2m1x8(x0);
-        c1 = e2m1x8(x1);
-      }
-      if (act) {
-        *reinterpret_cast<uint2 *>(data + row * (D / 2) + 8 * j) = make_uint2(c0, c1);
-        scales[row * (D / 16) + j] = static_cast<uint8_t>(sb_code);
-      }
+      c0 = e2m1x8(x0);
+      c1 = e2m1x8(x1);
+    }
+    if (act) {
+      *reinterpret_cast<uint2 *>(data + row * (D / 2) + 8 * j) = make_uint2(c0, c1);
+      scales[row * (D / 16) + j] = static_cast<uint8_t>(sb_code);
     }
   }
 }
