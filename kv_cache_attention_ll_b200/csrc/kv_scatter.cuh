@@ -12,11 +12,12 @@
 //            frame k of the held context (global sink, shot sink, window) to its
 //            slot (logical_slot)
 // Work split: the source rows ((token, head) pairs, D values each) are cut
-// into units of kRows rows of K and the same rows of V (8 KB of bf16 each), and
-// every CTA owns a contiguous range of units. A producer warp copies whole
-// units into shared memory with cp.async.bulk (one instruction per 8 KB,
-// completion counted on the stage's mbarrier), so each CTA has kStages units in
-// flight from its first clocks; eight consumer warps take a stage, convert its
+// into units of kRows rows of K and the same rows of V (8 KB of bf16 each for
+// an append, 16 KB for a recache), and every CTA owns a contiguous range of
+// units. A producer warp copies whole units into shared memory with
+// cp.async.bulk (one instruction per unit of K or V, completion counted on the
+// stage's mbarrier), so each CTA has kStages units in flight once it has read
+// the layer's counters; eight consumer warps take a stage, convert its
 // rows and store them to their planes, then hand the stage back. Everything
 // that depends on a layer's frame counters (the destination slot of a frame,
 // or that nothing is stored) is decided by the producer, once per unit.
