@@ -57,9 +57,10 @@ struct ScatterParams {
 };
 
 // Tile of the bulk scatter for head dimension D, with PASSES passes of the 8
-// consumer warps per unit: 8 KB units (6 stages) for the append, where the
-// launch is short and small units spread it over more CTAs, 16 KB units (3
-// stages) for the recache, a long stream where fewer, larger copies pay.
+// consumer warps per unit: 8 KB units (6 stages, 2 CTAs per SM) for the
+// append, where the launch is short and small units spread it over more CTAs;
+// 16 KB units (2 stages, 3 CTAs per SM) for the recache, a long stream where
+// fewer, larger copies and more converting warps per SM pay.
 template <int D, int PASSES>
 struct ScatterTile {
   static constexpr int kLPR = D / 16;                   // lanes per row, 16 values each
@@ -68,11 +69,13 @@ struct ScatterTile {
   static constexpr int kRows = kPasses * kPassRows;     // rows per unit
   static constexpr int kRowBytes = D * 2;               // one bf16 source row
   static constexpr int kUnitBytes = kRows * kRowBytes;  // kPasses x 8 KB of K (and as much of V)
-  static constexpr int kStages = 6 / kPasses;
+  static constexpr int kStages = PASSES == 2 ? 2 : 6;
+  static constexpr int kCtasPerSm = PASSES == 2 ? 3 : 2;
   static constexpr int kThreads = 288;                  // warps 0-7 consume, warp 8 produces
   // stages, then per stage a full and an empty barrier (8 bytes each) and a
-  // unit record (16 bytes), then the abort flag
-  static constexpr int kBookBytes = kStages * (8 + 8 + 16) + 16;
+  // unit record (16 bytes), then the abort flag (16 bytes), then the NVFP4
+  // reciprocal table (128 floats)
+  static constexpr int kBookBytes = kStages * (8 + 8 + 16) + 16 + 512;
   static constexpr int kSmem = kStages * 2 * kUnitBytes + kBookBytes;
   static_assert(kSmem <= 227 * 1024, "shared memory of one CTA");
 };
@@ -109,7 +112,7 @@ __device__ __forceinline__ uint32_t e4m3_code(float y) {
 // act = false take part in the shuffles and store nothing.
 template <int FMT, int D>
 __device__ __forceinline__ void store_row16(uint8_t *data, uint8_t *scales, long long row, int j, const uint4 &lo,
-                                            const uint4 &hi, bool act) {
+                                            const uint4 &hi, bool act, const float *rcp_tab) {
   constexpr int kLPR = D / 16;
   static_assert(FMT == FMT_FP8 || FMT == FMT_NVFP4, "quantised formats only");
   float x0[8], x1[8];
@@ -150,7 +153,7 @@ __device__ __forceinline__ void store_row16(uint8_t *data, uint8_t *scales, long
     const float sb = e4m3_to_f32(sb_code);
     uint32_t c0 = 0u, c1 = 0u;
     if (sb != 0.f) {
-      const float inv = __frcp_rn(sb);
+      const float inv = rcp_tab[sb_code];   // the correctly rounded 1 / sb
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         x0[e] = div_corrected(x0[e], sb, inv);
@@ -167,13 +170,14 @@ __device__ __forceinline__ void store_row16(uint8_t *data, uint8_t *scales, long
 }
 
 template <int FMT, int D, int PASSES>
-__global__ void __launch_bounds__(ScatterTile<D, PASSES>::kThreads, 2) kv_scatter_kernel(const ScatterParams q) {
+__global__ void __launch_bounds__(ScatterTile<D, PASSES>::kThreads, ScatterTile<D, PASSES>::kCtasPerSm) kv_scatter_kernel(const ScatterParams q) {
   using C = ScatterTile<D, PASSES>;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kStages * 2 * C::kUnitBytes);
   uint64_t *empty = full + C::kStages;
   int4 *unit_rec = reinterpret_cast<int4 *>(empty + C::kStages);   // (layer, slot or -1, first row, rows)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(unit_rec + C::kStages);
+  float *rcp_tab = reinterpret_cast<float *>(smem + C::kStages * 2 * C::kUnitBytes + C::kStages * 32 + 16);
 
   const int rows_frame = q.T * q.H;                               // source rows of one frame
   const int per_frame = (rows_frame + C::kRows - 1) / C::kRows;   // units of one frame
@@ -191,6 +195,10 @@ __global__ void __launch_bounds__(ScatterTile<D, PASSES>::kThreads, 2) kv_scatte
     }
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if constexpr (FMT == FMT_NVFP4) {
+    // 1 / sb for every E4M3 block-scale code (code 0 is never used as a divisor)
+    if (threadIdx.x < 128) rcp_tab[threadIdx.x] = threadIdx.x == 0 ? 0.f : __frcp_rn(e4m3_to_f32(threadIdx.x));
   }
   __syncthreads();
 
@@ -326,7 +334,7 @@ __global__ void __launch_bounds__(ScatterTile<D, PASSES>::kThreads, 2) kv_scatte
           const uint4 a = *reinterpret_cast<const uint4 *>(src + 16 * half_first);
           const uint4 c = *reinterpret_cast<const uint4 *>(src + 16 * (1 - half_first));
           store_row16<FMT, D>(q.data, q.scales, plane * q.slots + drow, j, half_first ? c : a, half_first ? a : c,
-                              act);
+                              act, rcp_tab);
         }
       }
     }

@@ -228,8 +228,8 @@ ll_status launch_scatter_kernel(const llk::ScatterParams &p, int device, cudaStr
   const long long units = static_cast<long long>(p.n_layers) * p.n_frames * ((rows_frame + C::kRows - 1) / C::kRows);
   if (units < 1 || units >= (1ll << 31)) return LL_ERR_INVALID_ARG;
   if (!prepare_scatter<FMT, D, PASSES>()) return LL_ERR_CUDA;
-  // two CTAs per SM, each owning a contiguous range of units (at least one)
-  long long grid = static_cast<long long>(num_sms(device)) * 2;
+  // kCtasPerSm CTAs per SM, each owning a contiguous range of units (at least one)
+  long long grid = static_cast<long long>(num_sms(device)) * C::kCtasPerSm;
   if (grid > units) grid = units;
   llk::kv_scatter_kernel<FMT, D, PASSES><<<static_cast<unsigned>(grid), C::kThreads, C::kSmem, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? LL_OK : LL_ERR_CUDA;
