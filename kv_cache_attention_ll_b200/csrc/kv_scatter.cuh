@@ -196,10 +196,6 @@ __global__ void __launch_bounds__(ScatterTile<D, PASSES>::kThreads, ScatterTile<
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if constexpr (FMT == FMT_NVFP4) {
-    // 1 / sb for every E4M3 block-scale code (code 0 is never used as a divisor)
-    if (threadIdx.x < 128) rcp_tab[threadIdx.x] = threadIdx.x == 0 ? 0.f : __frcp_rn(e4m3_to_f32(threadIdx.x));
-  }
   __syncthreads();
 
   if (warp == 8) {
@@ -297,6 +293,12 @@ __global__ void __launch_bounds__(ScatterTile<D, PASSES>::kThreads, ScatterTile<
   }
 
   // ---- consumers: warps 0-7, rows r0 + kPassRows * pass of each unit, 16 values per lane ----
+  if constexpr (FMT == FMT_NVFP4) {
+    // 1 / sb for every E4M3 block-scale code (code 0 is never a divisor), filled
+    // while the first copies are in flight; the eight warps alone meet here
+    if (threadIdx.x < 128) rcp_tab[threadIdx.x] = threadIdx.x == 0 ? 0.f : __frcp_rn(e4m3_to_f32(threadIdx.x));
+    named_bar_sync(1, 256);
+  }
   const int r0 = threadIdx.x / C::kLPR;
   const int j = threadIdx.x % C::kLPR;
   // the two 16-byte halves of a lane's 32 bytes are read in an order that puts
