@@ -97,6 +97,9 @@ typedef enum {
  *   head_dim in {64, 128}; sink_frames >= 0, window_frames >= 0,
  *   sink_frames + window_frames >= 1; (S+W)*T and F*T < 2^31; T*H*D/8 and
  *   (S+W)*T*D/8 < 2^30; heads < 32768.
+ *   The first cache created on a device also loads there every kernel a
+ *   chunk step can launch, so that no later call takes device memory for
+ *   kernel code (the footprint is fixed from here on).
  *   Returns LL_ERR_INVALID_ARG on a bad parameter or null `out`,
  *   LL_ERR_OOM if the allocation fails, LL_ERR_CUDA if no device is usable.
  *   On success *out owns the memory until ll_kv_cache_destroy.           */
